@@ -1,0 +1,405 @@
+"""Benchmark of the routed block-sparse attention path on B200.
+
+One step = one pass of the whole hot path over one layer of the chunk-48
+workload (40 heads, 48 query blocks, 2256 history blocks of 128 tokens,
+head_dim 128, bf16): Gilbert order + neighbour table, block importance, soft
+fusion and route build, routed attention.  Inputs are resident in HBM and
+larger than L2 (K + V = 5.9 GB), so no L2 flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl velox|reference]
+
+Prints one JSON line.  value = routed-attention FLOPs of the step (4 b^2 d per
+routed tile, from the actual route lengths) over the step time, summed over
+ranks (weak scaling: every rank runs its own layer; there is no data-path
+collective).  Per-call times, the roofline of the attention kernel, an
+end-to-end number through host buffers and the CPU oracle baseline are added.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "routed attn µs/call & TFLOP/s at chunk-48 shape; % of B200 bf16 peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LAUNCHES_PER_STEP = 7  # order, neighbours, pool, logits, softmax, route, attention
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            if self._t:
+                self._t.join(timeout=2)
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def _barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- oracle ---
+def cpu_oracle_sample(inp, attn_rows: int = 3, head: int = 0):
+    """Time the oracle on a bounded sample of one step and scale to a step.
+
+    Sample: importance of one head (all 48 x 2256 blocks), the routes of that
+    head's 48 rows, and attention of `attn_rows` rows of it.  The step
+    estimate multiplies each part by its share of the full step (40 heads,
+    1920 rows).
+    """
+    from oracle import attention as oatt
+    from oracle import gilbert as ogil
+    from oracle import importance as oimp
+    from oracle import route as ort
+    from threadpoolctl import threadpool_info
+
+    wl = inp.wl
+    H, N, M, b = wl.heads, wl.n_q_blocks, wl.n_kv_blocks, wl.b
+    prm = ort.Params(lam=wl.params.lam, tau=wl.params.tau, g_ref=wl.params.g_ref,
+                     theta_cov=wl.params.theta_cov, theta_unc=wl.params.theta_unc,
+                     k_cov=wl.params.k_cov, k_unc=wl.params.k_unc)
+    Qh = inp.Q[head].to(torch.float64).cpu().numpy()
+    Kh = inp.K[head].to(torch.float64).cpu().numpy()
+    Vh = inp.V[head].to(torch.float64).cpu().numpy()
+    g = inp.g.cpu().numpy()
+    cov = inp.covered.cpu().numpy()
+    t0 = time.perf_counter()
+    T, Hl, Wl = wl.lattice
+    nbr = ogil.neighbour_blocks(T, Hl, Wl, wl.n_chunks, b, wl.q_chunk, wl.cache_first_block, M)
+    t1 = time.perf_counter()
+    p = oimp.importance(Qh, Kh, b, 1.0).astype(np.float32)
+    t2 = time.perf_counter()
+    routes = [ort.route_row(p[i], g[i], bool(cov[i]), prm, wl.prev_begin, wl.prev_count, nbr[i])
+              for i in range(N)]
+    t3 = time.perf_counter()
+    flops = 0.0
+    for i in range(attn_rows):
+        tiles = routes[i][0] + routes[i][1]
+        oatt.routed_attention_block(Qh[i * b:(i + 1) * b], Kh, Vh, tiles, b)
+        flops += 4.0 * b * b * wl.d * len(tiles)
+    t4 = time.perf_counter()
+    step_s = (t1 - t0) + H * (t2 - t1) + H * (t3 - t2) + (H * N / attn_rows) * (t4 - t3)
+    threads = [x.get("num_threads", 1) for x in threadpool_info()
+               if x.get("user_api") == "blas"]
+    mean_len = float(np.mean([len(r[0]) + len(r[1]) for r in routes]))
+    return {"step_s": step_s, "sample_s": t4 - t0, "threads": max(threads) if threads else 1,
+            "mean_len": mean_len,
+            "sample": (f"Gilbert neighbour table; importance of head {head} (48x2256 blocks); "
+                       f"routes of its 48 rows; attention of {attn_rows} rows; scaled to a "
+                       f"step by 40 heads and {H * N} rows")}
+
+
+def run_reference(args, world, rank):
+    """--impl reference: the CPU oracle, on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    from synth import config, make_inputs
+    wl = config(3)
+    inp = make_inputs(wl, "cpu")
+    # FLOPs of the step: mean route length of the sampled head's oracle routes
+    times, flops_step = [], None
+    for s in range(args.warmup + args.steps):
+        r = cpu_oracle_sample(inp, attn_rows=2)
+        if s >= args.warmup:
+            times.append(r["step_s"])
+        if flops_step is None:
+            flops_step = 4.0 * 128 ** 3 * wl.heads * wl.n_q_blocks * r["mean_len"]
+    mean_s = sum(times) / len(times)
+    value = flops_step / mean_s / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": "chunk48 (H=40, N=48, M=2256, d=128, b_tok=128)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": r["threads"],
+                             "kind": "oracle", "sample": r["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- velox ---
+def run_velox(args, world, rank, local):
+    import routed_block_sparse_b200 as rbs
+    from routed_block_sparse_b200.pipeline import layer_for
+    from synth import config, make_inputs
+
+    dev = torch.device("cuda", local if world > 1 else 0)
+    wl = config(3, layer=rank)  # weak scaling: each rank its own layer
+    inp = make_inputs(wl, dev)
+    layer = layer_for(wl, device=dev)
+    H, N, M, b, d = wl.heads, wl.n_q_blocks, wl.n_kv_blocks, wl.b, wl.d
+    T, Hl, Wl = wl.lattice
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        rbs.velox_gilbert_order(T, Hl, Wl, wl.n_chunks, b, wl.q_chunk, wl.cache_first_block, M,
+                                nbr_ids=layer.nbr_ids, nbr_cnt=layer.nbr_cnt,
+                                S_max=layer.S_max, dev_status=layer.dev_status, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        layer.importance(inp.Q, inp.K, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        layer.route(inp.g, inp.covered, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        layer.attend(inp.Q, inp.K, inp.V, stream=stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    status = layer.status()
+    route_len = layer.route_len.to(torch.float64)
+    tiles = float(route_len.sum().item())
+    flops_step = 4.0 * b * b * d * tiles
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index or 0) as clocks:
+        t_start.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    _barrier(world)
+    torch.cuda.synchronize(dev)
+    total_ms = t_start.elapsed_time(t_end)
+    parts = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])
+    gil_ms, imp_ms, route_ms, attn_ms = parts.mean(axis=0)
+    ms_step = _max_over_ranks(total_ms / args.steps, world)
+    flops_all = _sum_over_ranks(flops_step, world)
+    value = flops_all / (ms_step * 1e-3) / 1e12
+
+    peaks, peak_kind = _peaks()
+    attn_tflops = flops_step / (attn_ms * 1e-3) / 1e12
+    imp_bytes = H * N * b * d * 2 + H * M * b * d * 2 + H * N * M * 4
+    route_bytes = (H * N * M * 4 + N * M * 4 + N + N * layer.S_max * 4 + N * 4
+                   + H * N * layer.R_max * 4 + 2 * H * N * 4)
+    imp_gbs = imp_bytes / (imp_ms * 1e-3) / 1e9
+    ir_gbs = (imp_bytes + route_bytes) / ((imp_ms + route_ms) * 1e-3) / 1e9
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if os.path.exists(tpath):
+        try:
+            with open(tpath) as f:
+                tj = json.load(f)
+            if tj.get("kernel_source_hash") == _attn_source_hash():
+                traffic = tj.get("bytes_per_launch")
+        except Exception:
+            traffic = None
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V; g U[0,1] half zeroed; coverage Bernoulli 0.5)",
+        "config": {"workload": "chunk48", "heads": H, "n_q_blocks": N, "n_kv_blocks": M,
+                   "head_dim": d, "b_tok": b, "k_cov": wl.params.k_cov, "k_unc": wl.params.k_unc,
+                   "theta": wl.params.theta_unc, "lattice": [T, Hl, Wl],
+                   "l2": "inputs larger than L2 (K+V 5.9 GB per layer), no flush"},
+        "attn_us": attn_ms * 1e3, "attn_tflops": attn_tflops,
+        "importance_us": imp_ms * 1e3, "importance_gbs": imp_gbs,
+        "route_us": route_ms * 1e3, "gilbert_us": gil_ms * 1e3,
+        "importance_route_gbs": ir_gbs, "importance_route_hbm_frac": ir_gbs / hbm,
+        "routed_tiles": tiles, "mean_route_len": tiles / (H * N), "dev_status": status,
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": bf16,
+                     "unit": "TFLOP/s", "frac": attn_tflops / bf16, "traffic": traffic,
+                     "peak_source": f"{peak_kind} bf16 dense (burst)"},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": clocks.summary(),
+    }
+
+    # end to end through the public API with host buffers
+    if args.e2e_steps > 0:
+        line["e2e"] = _e2e(args, wl, inp, layer, dev, stream, flops_step, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r = cpu_oracle_sample(inp)
+        line["cpu_baseline"] = {"value": flops_step / r["step_s"] / 1e12, "unit": UNIT,
+                                "cores": r["threads"], "kind": "oracle", "sample": r["sample"],
+                                "sample_seconds": r["sample_s"]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def _e2e(args, wl, inp, layer, dev, stream, flops_step, world):
+    """Per step: pinned host -> device copy of Q, K, V, g, covered; the four
+    calls; device -> host copy of O and lse.  Timed with CUDA events."""
+    host = {k: getattr(inp, k).cpu().pin_memory() for k in ("Q", "K", "V", "g", "covered")}
+    out_O = torch.empty_like(layer.O, device="cpu").pin_memory()
+    out_lse = torch.empty_like(layer.lse, device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_O.numel() * out_O.element_size() + out_lse.numel() * out_lse.element_size()
+    T, Hl, Wl = wl.lattice
+    import routed_block_sparse_b200 as rbs
+
+    def one():
+        for k, t in host.items():
+            getattr(inp, k).copy_(t, non_blocking=True)
+        rbs.velox_gilbert_order(T, Hl, Wl, wl.n_chunks, wl.b, wl.q_chunk, wl.cache_first_block,
+                                wl.n_kv_blocks, nbr_ids=layer.nbr_ids, nbr_cnt=layer.nbr_cnt,
+                                S_max=layer.S_max, dev_status=layer.dev_status, stream=stream)
+        layer.forward(inp.Q, inp.K, inp.V, inp.g, inp.covered, stream)
+        out_O.copy_(layer.O, non_blocking=True)
+        out_lse.copy_(layer.lse, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    z = torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        one()
+    z.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = _max_over_ranks(a.elapsed_time(z) / args.e2e_steps, world)
+    val = _sum_over_ranks(flops_step, world) / (ms * 1e-3) / 1e12
+    return {"value": val, "unit": UNIT, "ms_per_step": ms, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
+
+
+def _attn_source_hash() -> str:
+    import hashlib
+    p = os.path.join(ROOT, "routed_block_sparse_b200", "csrc", "attn.cu")
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="velox", choices=["velox", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = _dist_setup()
+    try:
+        run_velox(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

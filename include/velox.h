@@ -1,0 +1,241 @@
+/*
+ * velox.h -- C ABI of the B200 (sm_100a) routed block-sparse attention path.
+ *
+ * The path is the hot loop of Velox, a training-free router for the
+ * history attention of chunked video-diffusion world models ("Velox: Spatial
+ * Memory Makes Long-context World Models Efficient", project page
+ * velox-world.com, "02 · Method"; digest of arXiv 2610.22311 on
+ * paper.rainbus.top, "Core method" and "Method steps"):
+ *
+ *   1. velox_gilbert_order      global-aligned Gilbert token order, block ids,
+ *                               26-neighbour safeguard blocks;
+ *   2. velox_block_importance   p_{i,r} = softmax_r(scale * qbar_i . kbar_r);
+ *   3. velox_route_build        soft geometry fusion, minimal cumulative-mass
+ *                               prefix capped at K_cov / K_unc, reserved
+ *                               previous chunk, appended safeguards;
+ *   4. velox_block_sparse_attn  online-softmax attention over only the routed
+ *                               128-token KV tiles (tcgen05 / TMEM / TMA).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every pointer argument is a DEVICE pointer, owned by the caller, unless
+ *   the argument says "host".  The library never allocates, frees or keeps
+ *   caller memory; it keeps no state between calls except a per-device
+ *   cache of device attributes.
+ * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *   default stream) and may be issued from several host threads.
+ * - Tensors are dense and contiguous in the layouts stated.  bf16 values are
+ *   raw IEEE bfloat16 bit patterns (velox_bf16).
+ * - Host-detectable errors (null pointers, non-positive or inconsistent
+ *   sizes, unsupported head_dim / block size, too-small capacity or
+ *   workspace) return a status before anything is launched.  A CUDA launch
+ *   error returns VELOX_ERR_CUDA.
+ * - Errors that only the device can see (a route id out of range or
+ *   repeated, a capacity overflow, a bounded wait that gave up) are OR-ed
+ *   into *dev_status, one int32 in device memory that the caller zeroes
+ *   beforehand (VELOX_DEV_* bits).  The offending tile or row is skipped;
+ *   no kernel traps or reads out of bounds.
+ */
+#ifndef VELOX_H_
+#define VELOX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define VELOX_API __attribute__((visibility("default")))
+#else
+#define VELOX_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t velox_bf16;                 /* raw bfloat16 bits          */
+typedef struct CUstream_st *velox_stream_t;  /* == cudaStream_t            */
+
+typedef enum {
+  VELOX_OK = 0,
+  VELOX_ERR_INVALID_ARG = 1,  /* null pointer, bad size, inconsistent args */
+  VELOX_ERR_UNSUPPORTED = 2,  /* head_dim/block size/lattice not supported */
+  VELOX_ERR_WORKSPACE = 3,    /* workspace missing or too small            */
+  VELOX_ERR_CAPACITY = 4,     /* R_max / S_max cannot hold the output      */
+  VELOX_ERR_DEVICE = 5,       /* no usable sm_100 device                   */
+  VELOX_ERR_TIMEOUT = 6,      /* reserved: a bounded device wait gave up   */
+  VELOX_ERR_CUDA = 7          /* a CUDA runtime call or launch failed      */
+} velox_status;
+
+/* Bits OR-ed into *dev_status by the kernels. */
+#define VELOX_DEV_BAD_ROUTE_ID   0x01  /* route id < 0 or >= M: tile skipped   */
+#define VELOX_DEV_DUP_ROUTE_ID   0x02  /* id repeated in one route: skipped    */
+#define VELOX_DEV_ROUTE_LEN      0x04  /* route_len < 0 or > R_max: row zeroed */
+#define VELOX_DEV_NBR_OVERFLOW   0x08  /* more neighbours than S_max: cut      */
+#define VELOX_DEV_BAD_SAFEGUARD  0x10  /* nbr/ref id outside [0, M): ignored   */
+#define VELOX_DEV_WAIT_TIMEOUT   0x20  /* bounded mbarrier wait gave up        */
+#define VELOX_DEV_ROUTE_CAPACITY 0x40  /* route row longer than R_max: cut     */
+
+/* Supported sizes of the importance and attention calls. */
+#define VELOX_HEAD_DIM   128
+#define VELOX_BLOCK_TOK  128
+#define VELOX_MAX_BLOCKS 65536   /* max history blocks M per head            */
+#define VELOX_MAX_ROUTE  4096    /* max R_max (routed attention), k_cov, k_unc */
+
+/* Route hyper-parameters (onedev.kr summary, "How it differs": tau = 0.1,
+ * g_ref = 0.2, lambda = 2, K_cov = 80, K_unc = 150).  theta_* are the
+ * cumulative-mass thresholds of covered / uncovered rows (the pages give no
+ * value; 0.9 is the default of the bundled workloads). */
+typedef struct {
+  float lambda;     /* fusion strength; the multiplier is 1 + lambda * g^      */
+  float tau;        /* overlap noise floor: g^ = 0 unless g > tau              */
+  float g_ref;      /* overlap normaliser: g^ = min(g / g_ref, 1)              */
+  float theta_cov;  /* mass threshold, covered rows                            */
+  float theta_unc;  /* mass threshold, uncovered rows                          */
+  int32_t k_cov;    /* budget cap (reserved blocks included), covered rows     */
+  int32_t k_unc;    /* budget cap (reserved blocks included), uncovered rows   */
+} velox_route_params;
+
+/* Human-readable text of a status; never NULL. */
+VELOX_API const char *velox_status_string(velox_status s);
+
+/* ABI version of this header (major * 100 + minor). */
+VELOX_API int velox_abi_version(void);
+
+/*
+ * velox_gilbert_order -- global-aligned Gilbert order, block ids and the
+ * 26-neighbour safeguard table.
+ *
+ * Defined by: project page, "02 · Method", "Keeping neighbours adjacent in
+ * the block order" and figure "Incremental Gilbert order"; digest,
+ * "Prerequisites", "Gilbert space-filling curve", and "Method steps", Eq. 14.
+ *
+ * The lattice has n_chunks chunks of T latent frames of H x W tokens; global
+ * frame f = chunk * T + t; cell index c = (f * H + y) * W + x.  Each frame is
+ * walked by the 2-D generalised Hilbert (Gilbert) curve from (0,0) to
+ * (W-1,0), mirrored in x on odd global frames, frames in order:
+ *   rank(f, y, x) = f*H*W + r2[y][f odd ? W-1-x : x].
+ * Block id = rank / b_tok.  Requires W >= H, not (W odd and H even), and
+ * T*H*W % b_tok == 0 (blocks never straddle chunks); else UNSUPPORTED.
+ *
+ * Outputs (each nullable; int32, n_cells = n_chunks*T*H*W):
+ *   rank_of_cell[n_cells], cell_of_rank[n_cells], block_of_cell[n_cells].
+ * Safeguards of the N = T*H*W/b_tok query blocks of chunk q_chunk: history
+ * block u is listed for query block i when u != i, some token of u is within
+ * Chebyshev distance 1 of some token of i in (f, y, x), and
+ * cache_first_block <= u < cache_first_block + n_cache_blocks; it is written
+ * as the cache id u - cache_first_block.  nbr_ids[N][S_max] (ascending, -1
+ * padded) and nbr_cnt[N]; both null to skip.  More than S_max neighbours:
+ * the S_max lowest are kept and VELOX_DEV_NBR_OVERFLOW is set.
+ * dev_status may be null only when nbr_ids is null.
+ */
+VELOX_API velox_status velox_gilbert_order(int T, int H, int W, int n_chunks, int b_tok,
+                                 int q_chunk, int cache_first_block,
+                                 int n_cache_blocks, int32_t *rank_of_cell,
+                                 int32_t *cell_of_rank, int32_t *block_of_cell,
+                                 int32_t *nbr_ids, int32_t *nbr_cnt, int S_max,
+                                 int32_t *dev_status, velox_stream_t stream);
+
+/*
+ * velox_workspace_size -- bytes of device workspace that
+ * velox_block_importance and velox_route_build need for these sizes
+ * (one buffer serves both; 256-byte aligned).  bytes: host pointer.
+ */
+VELOX_API velox_status velox_workspace_size(int H, int N, int M, int d, size_t *bytes);
+
+/*
+ * velox_block_importance -- per-head block importance.
+ *
+ * Defined by: digest, "Method steps", step four (Eq. 9); onedev.kr summary,
+ * "How it differs"; project page, "02 · Method", glossary entry for p.
+ *
+ *   qbar[h][i] = mean of the b_tok query tokens of block i   (fp32 accum.)
+ *   kbar[h][r] = mean of the b_tok key tokens of block r
+ *   p[h][i][r] = exp(l_r - max_r l) / sum_r exp(l_r - max_r l),
+ *                l_r = scale * qbar[h][i] . kbar[h][r]
+ *
+ * Q [H][N*b_tok][d] bf16, K [H][M*b_tok][d] bf16 (Gilbert token order,
+ * head-major), p [H][N][M] fp32 out.  d == b_tok == 128.  ws: device
+ * workspace of at least velox_workspace_size() bytes.
+ */
+VELOX_API velox_status velox_block_importance(const velox_bf16 *Q, const velox_bf16 *K,
+                                    int H, int N, int M, int d, int b_tok,
+                                    float scale, float *p, void *ws,
+                                    size_t ws_bytes, velox_stream_t stream);
+
+/*
+ * velox_route_build -- soft geometry fusion and route materialisation.
+ *
+ * Defined by: project page, "02 · Method", fusion formula
+ * p~ ~ p (1 + lambda g^), g^ = [g > tau] min(g / g_ref, 1), and "Covered and
+ * uncovered blocks"; digest, "Core method" (Eq. 11) and "Method steps"
+ * (Eq. 12-14); onedev.kr summary, "How it differs".
+ *
+ * Per row (h, i):
+ *   w_r = covered[i] ? p_r (1 + lambda g^_{i,r}) : p_r        (fp64)
+ *   s_r = covered[i] ? w_r / sum_r' w_r' : p_r                 (fp64)
+ *   walk: reserved blocks [prev_begin, prev_begin+prev_count) first, then
+ *   the others by w descending (ties: lower id); take blocks while
+ *   count < K (K_cov / K_unc) and cumulative s < theta (theta_cov /
+ *   theta_unc); reserved blocks are always taken.
+ *   extras = (nbr_ids[i][0..nbr_cnt[i]) U ref_ids) minus the budget.
+ * Output row: the budget ids ascending, then the extras ascending, each id
+ * once; route_len[h][i] = total, route_nbudget[h][i] = budget count; the
+ * rest of the row is -1.
+ *
+ * p [H][N][M] fp32, g [N][M] fp32 (shared by all heads), covered [N] uint8,
+ * nbr_ids [N][S_max] / nbr_cnt [N] int32 (both null, or S_max = 0, for no
+ * neighbours), ref_ids [n_ref] int32 (null when n_ref = 0).
+ * route_ids [H][N][R_max] int32, route_len / route_nbudget [H][N] int32.
+ * R_max must be >= min(M, max(k_cov, k_unc, prev_count) + S_max + n_ref);
+ * 0 <= k_cov, k_unc <= VELOX_MAX_ROUTE; M <= VELOX_MAX_BLOCKS.  p must be
+ * finite and non-negative.
+ * Safeguard ids outside [0, M) are ignored and flag VELOX_DEV_BAD_SAFEGUARD.
+ * ws: device workspace of at least velox_workspace_size() bytes.
+ */
+VELOX_API velox_status velox_route_build(const float *p, const float *g,
+                               const uint8_t *covered,
+                               const velox_route_params *prm, /* host */
+                               int prev_begin, int prev_count,
+                               const int32_t *nbr_ids, const int32_t *nbr_cnt,
+                               int S_max, const int32_t *ref_ids, int n_ref,
+                               int H, int N, int M, int32_t *route_ids,
+                               int32_t *route_len, int32_t *route_nbudget,
+                               int R_max, void *ws, size_t ws_bytes,
+                               int32_t *dev_status, velox_stream_t stream);
+
+/*
+ * velox_block_sparse_attn -- attention over routed KV tiles.
+ *
+ * Defined by: digest, "Core method" (Eq. 15) and "Novelty"; project page,
+ * "Why the route is a block, not a token"; onedev.kr summary, "How to use".
+ *
+ * For head h, query block i and each of its b_tok query tokens q:
+ *   O[h][i*b+t] = sum_u softmax_u(softmax_scale * q . k_u) v_u
+ * over the tokens u of the tiles route_ids[h][i][0 .. route_len[h][i]),
+ * tile r covering key/value tokens [r*b_tok, (r+1)*b_tok) of head h.
+ * lse[h][i*b+t] = log sum_u exp(softmax_scale * q . k_u) (natural log).
+ * An empty route gives O = 0 and lse = -inf.  route_ids == NULL computes
+ * dense attention over all M tiles (route_len ignored).
+ *
+ * Q [H][N*b][d], K and V [H][M*b][d] bf16; O [H][N*b][d] bf16 out;
+ * lse [H][N*b] fp32 out (nullable).  softmax_scale <= 0 means 1/sqrt(d).
+ * d == b_tok == 128, M <= VELOX_MAX_BLOCKS, R_max <= VELOX_MAX_ROUTE when
+ * routed.  A route id outside [0, M) or
+ * repeated within its row is skipped (VELOX_DEV_BAD_ROUTE_ID /
+ * VELOX_DEV_DUP_ROUTE_ID); route_len outside [0, R_max] zeroes the row
+ * (VELOX_DEV_ROUTE_LEN).  Q, K, V, O must be 16-byte aligned.
+ */
+VELOX_API velox_status velox_block_sparse_attn(const velox_bf16 *Q, const velox_bf16 *K,
+                                     const velox_bf16 *V,
+                                     const int32_t *route_ids,
+                                     const int32_t *route_len, int R_max,
+                                     int H, int N, int M, int d, int b_tok,
+                                     float softmax_scale, velox_bf16 *O,
+                                     float *lse, int32_t *dev_status,
+                                     velox_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VELOX_H_ */

@@ -1,0 +1,254 @@
+// Global-aligned Gilbert order and 26-neighbour safeguard blocks.
+//
+// Velox project page, "02 · Method", "Keeping neighbours adjacent in the
+// block order" and figure "Incremental Gilbert order": the KV cache is stored
+// in a Gilbert space-filling order, built once per frame and mirrored on
+// alternate frames so that frame and chunk seams stay adjacent; 128-token
+// blocks of that order are the route ids, and lattice neighbours of a query
+// block are safeguards (digest of arXiv 2610.22311, "Method steps", Eq. 14).
+//
+// Instead of generating the curve sequentially, every thread locates its own
+// cell by descending the generalised-Hilbert recursion: at each level the
+// rectangle is cut into two (long rectangles) or three pieces, the piece
+// holding the cell is found by a containment test, and the sizes of the
+// pieces walked before it are added to the rank.  The depth is O(log(WH)).
+// The inverse (rank -> cell) descends the same recursion by piece sizes.
+#include "common.cuh"
+
+namespace velox {
+namespace {
+
+struct Rect {
+  int x, y;    // start corner
+  int ax, ay;  // major edge vector
+  int bx, by;  // minor edge vector
+};
+
+__device__ __forceinline__ int sgn(int v) { return (v > 0) - (v < 0); }
+// floor(v / 2) for negative v as well (the recursion halves signed vectors)
+__device__ __forceinline__ int floor_half(int v) { return (v - (v & 1)) / 2; }
+__device__ __forceinline__ int iabs(int v) { return v < 0 ? -v : v; }
+
+__device__ __forceinline__ bool contains(const Rect &r, int cx, int cy) {
+  int ux = sgn(r.ax), uy = sgn(r.ay), vx = sgn(r.bx), vy = sgn(r.by);
+  int i = (cx - r.x) * ux + (cy - r.y) * uy;
+  int j = (cx - r.x) * vx + (cy - r.y) * vy;
+  return i >= 0 && i < iabs(r.ax + r.ay) && j >= 0 && j < iabs(r.bx + r.by);
+}
+
+// The pieces of one recursion level.  Returns the number of pieces (2 or 3)
+// or 0 for a one-cell-thick rectangle (a straight line).
+__device__ __forceinline__ int split(const Rect &r, Rect (&p)[3]) {
+  int nmaj = iabs(r.ax + r.ay), nmin = iabs(r.bx + r.by);
+  if (nmin == 1 || nmaj == 1) return 0;
+  int ux = sgn(r.ax), uy = sgn(r.ay), vx = sgn(r.bx), vy = sgn(r.by);
+  int hax = floor_half(r.ax), hay = floor_half(r.ay);
+  int hbx = floor_half(r.bx), hby = floor_half(r.by);
+  if (2 * nmaj > 3 * nmin) {
+    if ((iabs(hax + hay) & 1) && nmaj > 2) { hax += ux; hay += uy; }
+    p[0] = {r.x, r.y, hax, hay, r.bx, r.by};
+    p[1] = {r.x + hax, r.y + hay, r.ax - hax, r.ay - hay, r.bx, r.by};
+    return 2;
+  }
+  if ((iabs(hbx + hby) & 1) && nmin > 2) { hbx += vx; hby += vy; }
+  p[0] = {r.x, r.y, hbx, hby, hax, hay};
+  p[1] = {r.x + hbx, r.y + hby, r.ax, r.ay, r.bx - hbx, r.by - hby};
+  p[2] = {r.x + (r.ax - ux) + (hbx - vx), r.y + (r.ay - uy) + (hby - vy), -hbx, -hby,
+          -(r.ax - hax), -(r.ay - hay)};
+  return 3;
+}
+
+__device__ __forceinline__ int area(const Rect &r) {
+  return iabs(r.ax + r.ay) * iabs(r.bx + r.by);
+}
+
+// Position of cell (cx, cy) on the curve of a W x H frame (W >= H).
+__device__ int frame_rank(int W, int H, int cx, int cy) {
+  Rect r = {0, 0, W, 0, 0, H};
+  int base = 0;
+  for (;;) {
+    Rect p[3];
+    int n = split(r, p);
+    if (n == 0) {
+      // a line: along the major edge if it is one cell thick, else the minor
+      if (iabs(r.bx + r.by) == 1)
+        return base + (cx - r.x) * sgn(r.ax) + (cy - r.y) * sgn(r.ay);
+      return base + (cx - r.x) * sgn(r.bx) + (cy - r.y) * sgn(r.by);
+    }
+    int k = 0;
+    while (k < n - 1 && !contains(p[k], cx, cy)) {
+      base += area(p[k]);
+      ++k;
+    }
+    r = p[k];
+  }
+}
+
+// Cell at position k of the curve of a W x H frame.
+__device__ void frame_cell(int W, int H, int k, int &cx, int &cy) {
+  Rect r = {0, 0, W, 0, 0, H};
+  for (;;) {
+    Rect p[3];
+    int n = split(r, p);
+    if (n == 0) {
+      if (iabs(r.bx + r.by) == 1) {
+        cx = r.x + k * sgn(r.ax);
+        cy = r.y + k * sgn(r.ay);
+      } else {
+        cx = r.x + k * sgn(r.bx);
+        cy = r.y + k * sgn(r.by);
+      }
+      return;
+    }
+    int q = 0;
+    while (q < n - 1 && k >= area(p[q])) {
+      k -= area(p[q]);
+      ++q;
+    }
+    r = p[q];
+  }
+}
+
+struct Lattice {
+  int T, H, W, n_chunks, b;
+  __device__ int HW() const { return H * W; }
+  // global rank of cell (f, y, x)
+  __device__ int rank(int f, int y, int x) const {
+    int xm = (f & 1) ? (W - 1 - x) : x;
+    return f * H * W + frame_rank(W, H, xm, y);
+  }
+};
+
+__global__ void order_kernel(Lattice L, int n_cells, int32_t *rank_of_cell,
+                             int32_t *cell_of_rank, int32_t *block_of_cell) {
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < n_cells; c += gridDim.x * blockDim.x) {
+    int f = c / L.HW();
+    int rem = c - f * L.HW();
+    int y = rem / L.W;
+    int x = rem - y * L.W;
+    int r = L.rank(f, y, x);
+    if (rank_of_cell) rank_of_cell[c] = r;
+    if (cell_of_rank) cell_of_rank[r] = c;
+    if (block_of_cell) block_of_cell[c] = r / L.b;
+  }
+}
+
+// One CTA per query block of chunk q_chunk.  Candidates (26 offsets of each
+// of the b tokens) are gathered in shared memory, sorted, deduplicated.
+__global__ void neighbour_kernel(Lattice L, int q_chunk, int cache_first, int n_cache,
+                                 int32_t *nbr_ids, int32_t *nbr_cnt, int S_max, int cap,
+                                 int32_t *dev_status) {
+  extern __shared__ int cand[];  // cap entries (a power of two)
+  __shared__ int s_count;
+  __shared__ int s_scan[1024];
+  const int per_chunk = L.T * L.H * L.W / L.b;
+  const int i = blockIdx.x;
+  const int qb = q_chunk * per_chunk + i;
+  for (int k = threadIdx.x; k < cap; k += blockDim.x) cand[k] = INT32_MAX;
+  if (threadIdx.x == 0) s_count = 0;
+  __syncthreads();
+  const int HW = L.HW();
+  const int F = L.n_chunks * L.T;
+  for (int t = threadIdx.x; t < L.b; t += blockDim.x) {
+    int rank = qb * L.b + t;
+    int f = rank / HW;
+    int k = rank - f * HW;
+    int xm, y;
+    frame_cell(L.W, L.H, k, xm, y);
+    int x = (f & 1) ? (L.W - 1 - xm) : xm;
+    for (int o = 0; o < 27; ++o) {
+      if (o == 13) continue;  // the centre
+      int f2 = f + o / 9 - 1, y2 = y + (o / 3) % 3 - 1, x2 = x + o % 3 - 1;
+      if (f2 < 0 || f2 >= F || y2 < 0 || y2 >= L.H || x2 < 0 || x2 >= L.W) continue;
+      int u = L.rank(f2, y2, x2) / L.b;
+      if (u == qb || u < cache_first || u >= cache_first + n_cache) continue;
+      int slot = atomicAdd(&s_count, 1);
+      cand[slot] = u - cache_first;  // slot < 26 * b <= cap by construction
+    }
+  }
+  __syncthreads();
+  // bitonic sort of cap entries (INT32_MAX padding sorts last)
+  for (int size = 2; size <= cap; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int k = threadIdx.x; k < cap; k += blockDim.x) {
+        int partner = k ^ stride;
+        if (partner > k) {
+          bool up = ((k & size) == 0);
+          int a = cand[k], b2 = cand[partner];
+          if ((a > b2) == up) {
+            cand[k] = b2;
+            cand[partner] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // keep the first of each run of equal ids: ordered compaction, thread t
+  // owning a contiguous chunk of the sorted array
+  const int n = s_count;
+  const int chunk = (n + blockDim.x - 1) / blockDim.x;
+  const int lo = threadIdx.x * chunk, hi = min(n, lo + chunk);
+  int mine = 0;
+  for (int k = lo; k < hi; ++k) mine += (k == 0 || cand[k] != cand[k - 1]);
+  s_scan[threadIdx.x] = mine;
+  __syncthreads();
+  for (int off = 1; off < (int)blockDim.x; off <<= 1) {
+    int v = threadIdx.x >= (unsigned)off ? s_scan[threadIdx.x - off] : 0;
+    __syncthreads();
+    s_scan[threadIdx.x] += v;
+    __syncthreads();
+  }
+  const int total = s_scan[blockDim.x - 1];
+  int pos = s_scan[threadIdx.x] - mine;
+  for (int k = lo; k < hi; ++k) {
+    if (k == 0 || cand[k] != cand[k - 1]) {
+      if (pos < S_max && nbr_ids) nbr_ids[(size_t)i * S_max + pos] = cand[k];
+      ++pos;
+    }
+  }
+  for (int k = total + threadIdx.x; k < S_max; k += blockDim.x)
+    if (nbr_ids) nbr_ids[(size_t)i * S_max + k] = -1;
+  if (threadIdx.x == 0) {
+    if (nbr_cnt) nbr_cnt[i] = min(total, S_max);
+    if (total > S_max) flag_error(dev_status, VELOX_DEV_NBR_OVERFLOW);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gilbert(int T, int H, int W, int n_chunks, int b, int q_chunk,
+                           int cache_first, int n_cache, int32_t *rank_of_cell,
+                           int32_t *cell_of_rank, int32_t *block_of_cell, int32_t *nbr_ids,
+                           int32_t *nbr_cnt, int S_max, int32_t *dev_status,
+                           cudaStream_t stream) {
+  Lattice L{T, H, W, n_chunks, b};
+  const int n_cells = n_chunks * T * H * W;
+  if (rank_of_cell || cell_of_rank || block_of_cell) {
+    int grid = (n_cells + 255) / 256;
+    if (grid > 148 * 32) grid = 148 * 32;
+    order_kernel<<<grid, 256, 0, stream>>>(L, n_cells, rank_of_cell, cell_of_rank,
+                                           block_of_cell);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (nbr_ids || nbr_cnt) {
+    int cap = 1;
+    while (cap < 26 * b) cap <<= 1;
+    const int per_chunk = T * H * W / b;
+    size_t smem = (size_t)cap * sizeof(int);
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(neighbour_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    neighbour_kernel<<<per_chunk, 256, smem, stream>>>(L, q_chunk, cache_first, n_cache,
+                                                       nbr_ids, nbr_cnt, S_max, cap,
+                                                       dev_status);
+    return cudaGetLastError();
+  }
+  return cudaSuccess;
+}
+
+}  // namespace velox

@@ -1,0 +1,208 @@
+// Per-head block importance p_{i,r} = softmax_r(scale * qbar_i . kbar_r).
+//
+// Digest of arXiv 2610.22311, "Method steps", step four (Eq. 9); onedev.kr
+// summary, "How it differs": each layer's block importance is the softmax of
+// the mean-query / mean-key inner product.
+//
+// Three launches:
+//   pool_kernel     streams Q and K once (the HBM-bound part: at the
+//                   chunk-48 shape K alone is 2.96 GB) and writes the fp32
+//                   block means qbar [H][N][d], kbar [H][M][d] to the
+//                   workspace.  One warp per 128 x 128 bf16 block, 16-byte
+//                   non-caching loads, 8 loads in flight per lane.
+//   logits_kernel   per (head, 64 history blocks): the N x 64 tile of
+//                   scale * qbar . kbar, written into p as raw logits.
+//   softmax_kernel  per (head, query block) row: max, sum of exp, normalise.
+#include "common.cuh"
+
+namespace velox {
+namespace {
+
+constexpr int D = VELOX_HEAD_DIM;
+constexpr int BT = VELOX_BLOCK_TOK;
+
+__device__ __forceinline__ uint4 ld_stream(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void acc8(float (&a)[8], const uint4 &v) {
+  a[0] += bf16_lo(v.x); a[1] += bf16_hi(v.x);
+  a[2] += bf16_lo(v.y); a[3] += bf16_hi(v.y);
+  a[4] += bf16_lo(v.z); a[5] += bf16_hi(v.z);
+  a[6] += bf16_lo(v.w); a[7] += bf16_hi(v.w);
+}
+
+// Unit u < n_q: query block (h = u / N, i = u % N); else key block.
+// Rows of a block are 256 bytes = 16 lanes x 16 bytes: lanes 0-15 take even
+// rows, lanes 16-31 odd rows; each lane sums 8 channels over 64 rows.
+__global__ void __launch_bounds__(256) pool_kernel(const uint16_t *__restrict__ Q,
+                                                   const uint16_t *__restrict__ K, int n_q,
+                                                   int n_units, float *__restrict__ qbar,
+                                                   float *__restrict__ kbar) {
+  const int lane = threadIdx.x & 31;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int n_warps = (gridDim.x * blockDim.x) >> 5;
+  const int col = (lane & 15) * 8;
+  const int row0 = lane >> 4;
+  for (int u = warp; u < n_units; u += n_warps) {
+    const uint16_t *src;
+    float *dst;
+    if (u < n_q) {
+      src = Q + (size_t)u * BT * D;
+      dst = qbar + (size_t)u * D;
+    } else {
+      src = K + (size_t)(u - n_q) * BT * D;
+      dst = kbar + (size_t)(u - n_q) * D;
+    }
+    float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const uint16_t *p = src + row0 * D + col;
+#pragma unroll 1
+    for (int r = 0; r < BT / 2; r += 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = ld_stream(p + (size_t)(r + k) * 2 * D);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc8(a, v[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] += __shfl_xor_sync(0xffffffffu, a[k], 16);
+    if (lane < 16) {
+      const float inv = 1.0f / BT;
+      float4 lo = make_float4(a[0] * inv, a[1] * inv, a[2] * inv, a[3] * inv);
+      float4 hi = make_float4(a[4] * inv, a[5] * inv, a[6] * inv, a[7] * inv);
+      reinterpret_cast<float4 *>(dst + col)[0] = lo;
+      reinterpret_cast<float4 *>(dst + col)[1] = hi;
+    }
+  }
+}
+
+// Logit tile: 64 history blocks per CTA, query rows 16 at a time.  The key
+// means are stored transposed (channel-major) so that thread tx reads the
+// 4 blocks 4*tx .. 4*tx+3 of one channel as a single float4; thread ty owns
+// one query row of the current group.
+constexpr int LG_R = 64;   // history blocks per CTA
+constexpr int LG_Q = 16;   // query rows per pass
+
+__global__ void __launch_bounds__(256) logits_kernel(const float *__restrict__ qbar,
+                                                     const float *__restrict__ kbar, int N,
+                                                     int M, float scale, float *__restrict__ p) {
+  __shared__ __align__(16) float ks[D][LG_R + 4];
+  __shared__ float qs[LG_Q][D + 4];
+  const int h = blockIdx.y;
+  const int r0 = blockIdx.x * LG_R;
+  const int tid = threadIdx.x;
+  const float *kb = kbar + ((size_t)h * M + r0) * D;
+  for (int e = tid; e < LG_R * D / 4; e += blockDim.x) {
+    int r = e / (D / 4), c = (e % (D / 4)) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r0 + r < M) v = *reinterpret_cast<const float4 *>(kb + (size_t)r * D + c);
+    ks[c][r] = v.x; ks[c + 1][r] = v.y; ks[c + 2][r] = v.z; ks[c + 3][r] = v.w;
+  }
+  const int ty = tid >> 4, tx = tid & 15;
+  for (int i0 = 0; i0 < N; i0 += LG_Q) {
+    __syncthreads();
+    for (int e = tid; e < LG_Q * D / 4; e += blockDim.x) {
+      int r = e / (D / 4), c = (e % (D / 4)) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i0 + r < N)
+        v = *reinterpret_cast<const float4 *>(qbar + ((size_t)h * N + i0 + r) * D + c);
+      qs[r][c] = v.x; qs[r][c + 1] = v.y; qs[r][c + 2] = v.z; qs[r][c + 3] = v.w;
+    }
+    __syncthreads();
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int c = 0; c < D; ++c) {
+      const float q = qs[ty][c];
+      const float4 k4 = *reinterpret_cast<const float4 *>(&ks[c][4 * tx]);
+      acc.x = fmaf(q, k4.x, acc.x);
+      acc.y = fmaf(q, k4.y, acc.y);
+      acc.z = fmaf(q, k4.z, acc.z);
+      acc.w = fmaf(q, k4.w, acc.w);
+    }
+    const int i = i0 + ty;
+    if (i < N) {
+      float *dst = p + ((size_t)h * N + i) * M + r0 + 4 * tx;
+      const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (r0 + 4 * tx + k < M) dst[k] = scale * v[k];
+    }
+  }
+}
+
+__device__ __forceinline__ void merge_ms(float &m, float &s, float m2, float s2) {
+  float mm = fmaxf(m, m2);
+  if (mm == -INFINITY) return;
+  s = s * expf(m - mm) + s2 * expf(m2 - mm);
+  m = mm;
+}
+
+// One CTA per (h, i) row of M logits, in place.
+__global__ void __launch_bounds__(256) softmax_kernel(float *__restrict__ p, int M) {
+  __shared__ float sm[8], ss[8];
+  float *row = p + (size_t)blockIdx.x * M;
+  float m = -INFINITY, s = 0.f;
+  for (int r = threadIdx.x; r < M; r += blockDim.x) {
+    float x = row[r];
+    if (x > m) {
+      s = s * expf(m - x) + 1.0f;
+      m = x;
+    } else {
+      s += expf(x - m);
+    }
+  }
+  for (int off = 16; off > 0; off >>= 1) {
+    float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+    float s2 = __shfl_xor_sync(0xffffffffu, s, off);
+    merge_ms(m, s, m2, s2);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) { sm[warp] = m; ss[warp] = s; }
+  __syncthreads();
+  if (warp == 0) {
+    int nw = blockDim.x >> 5;
+    m = lane < nw ? sm[lane] : -INFINITY;
+    s = lane < nw ? ss[lane] : 0.f;
+    for (int off = 16; off > 0; off >>= 1) {
+      float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+      float s2 = __shfl_xor_sync(0xffffffffu, s, off);
+      merge_ms(m, s, m2, s2);
+    }
+    if (lane == 0) { sm[0] = m; ss[0] = s; }
+  }
+  __syncthreads();
+  const float gm = sm[0], inv = 1.0f / ss[0];
+  for (int r = threadIdx.x; r < M; r += blockDim.x) row[r] = expf(row[r] - gm) * inv;
+}
+
+}  // namespace
+
+size_t importance_workspace_bytes(int H, int N, int M) {
+  size_t b = (size_t)H * ((size_t)N + (size_t)M) * D * sizeof(float);
+  return (b + 255) & ~(size_t)255;
+}
+
+cudaError_t launch_importance(const uint16_t *Q, const uint16_t *K, int H, int N, int M,
+                              float scale, float *p, void *ws, cudaStream_t stream) {
+  float *qbar = static_cast<float *>(ws);
+  float *kbar = qbar + (size_t)H * N * D;
+  const int n_q = H * N;
+  const int n_units = H * (N + M);
+  int grid = (n_units + 7) / 8;
+  if (grid > 148 * 8 * 4) grid = 148 * 8 * 4;
+  pool_kernel<<<grid, 256, 0, stream>>>(Q, K, n_q, n_units, qbar, kbar);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dim3 lg((M + LG_R - 1) / LG_R, H);
+  logits_kernel<<<lg, 256, 0, stream>>>(qbar, kbar, N, M, scale, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  softmax_kernel<<<H * N, 256, 0, stream>>>(p, M);
+  return cudaGetLastError();
+}
+
+}  // namespace velox

@@ -1,0 +1,66 @@
+"""GPU block importance vs the oracle (fp32 vs fp64, relative tolerance)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from synth import config, make_inputs
+from synth.configs import small
+from parity import P_RTOL, f64, oracle_importance
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(lib, inp, scale):
+    wl = inp.wl
+    H, N, M = wl.heads, wl.n_q_blocks, wl.n_kv_blocks
+    p = torch.full((H, N, M), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.empty(lib.velox_workspace_size(H, N, M), dtype=torch.uint8, device="cuda")
+    lib.velox_block_importance(inp.Q, inp.K, H, N, M, 128, 128, scale, p, ws)
+    torch.cuda.synchronize()
+    return p
+
+
+def _check(p, ref):
+    for h, ph in ref.items():
+        g = f64(p[h])
+        assert np.all(np.isfinite(g))
+        rel = np.abs(g / ph - 1.0).max()
+        assert rel <= P_RTOL, f"head {h}: rel err {rel}"
+        assert abs(g.sum(axis=1) - 1.0).max() < 1e-4
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
+@pytest.mark.parametrize("scale", [1.0, 1.0 / math.sqrt(128)])
+def test_importance_small_configs(lib, cfg, scale):
+    inp = make_inputs(config(cfg), "cuda")
+    p = _run(lib, inp, scale)
+    _check(p, oracle_importance(inp.Q, inp.K, range(inp.wl.heads), scale))
+
+
+@pytest.mark.slow
+def test_importance_chunk48_sampled_heads(lib):
+    inp = make_inputs(config(3), "cuda")
+    p = _run(lib, inp, 1.0)
+    _check(p, oracle_importance(inp.Q, inp.K, [0, 17, 39], 1.0))
+
+
+@pytest.mark.parametrize("H,N,M", [(1, 1, 1), (2, 3, 65), (3, 17, 130), (1, 40, 200)])
+def test_importance_ragged_shapes(lib, H, N, M):
+    inp = make_inputs(small(H, N, M, 0), "cuda")
+    p = _run(lib, inp, 1.0)
+    _check(p, oracle_importance(inp.Q, inp.K, range(H), 1.0))
+
+
+def test_importance_peaked_logits(lib):
+    # large scale: rows nearly one-hot, still relative-accurate on the mass
+    inp = make_inputs(small(2, 4, 50, 0, key_mean_sigma=2.0), "cuda")
+    p = _run(lib, inp, 8.0)
+    ref = oracle_importance(inp.Q, inp.K, range(2), 8.0)
+    for h, ph in ref.items():
+        g = f64(p[h])
+        big = ph > 1e-6
+        assert np.abs(g[big] / ph[big] - 1.0).max() <= 50 * P_RTOL
+        assert np.abs(g - ph).max() < 1e-6
