@@ -142,13 +142,13 @@ def _sum_over_ranks(x: float, world: int) -> float:
 
 
 # ---------------------------------------------------------------- oracle ---
-def cpu_oracle_sample(inp, attn_rows: int = 3, head: int = 0):
+def cpu_oracle_sample(inp, attn_rows: int = 48, heads=(0, 1, 2, 3)):
     """Time the oracle on a bounded sample of one step and scale to a step.
 
-    Sample: importance of one head (all 48 x 2256 blocks), the routes of that
-    head's 48 rows, and attention of `attn_rows` rows of it.  The step
-    estimate multiplies each part by its share of the full step (40 heads,
-    1920 rows).
+    Sample: the neighbour table, importance of `heads` (all 48 x 2256 blocks
+    each), the routes of their rows, and attention of `attn_rows` rows of
+    the first of them.  The step estimate multiplies each part by its share
+    of the full step (40 heads, 1920 rows).
     """
     from oracle import attention as oatt
     from oracle import gilbert as ogil
@@ -161,35 +161,38 @@ def cpu_oracle_sample(inp, attn_rows: int = 3, head: int = 0):
     prm = ort.Params(lam=wl.params.lam, tau=wl.params.tau, g_ref=wl.params.g_ref,
                      theta_cov=wl.params.theta_cov, theta_unc=wl.params.theta_unc,
                      k_cov=wl.params.k_cov, k_unc=wl.params.k_unc)
-    Qh = inp.Q[head].to(torch.float64).cpu().numpy()
-    Kh = inp.K[head].to(torch.float64).cpu().numpy()
-    Vh = inp.V[head].to(torch.float64).cpu().numpy()
+    Qs = {h: inp.Q[h].to(torch.float64).cpu().numpy() for h in heads}
+    Ks = {h: inp.K[h].to(torch.float64).cpu().numpy() for h in heads}
+    Vh = inp.V[heads[0]].to(torch.float64).cpu().numpy()
     g = inp.g.cpu().numpy()
     cov = inp.covered.cpu().numpy()
     t0 = time.perf_counter()
     T, Hl, Wl = wl.lattice
     nbr = ogil.neighbour_blocks(T, Hl, Wl, wl.n_chunks, b, wl.q_chunk, wl.cache_first_block, M)
     t1 = time.perf_counter()
-    p = oimp.importance(Qh, Kh, b, 1.0).astype(np.float32)
+    p = {h: oimp.importance(Qs[h], Ks[h], b, 1.0).astype(np.float32) for h in heads}
     t2 = time.perf_counter()
-    routes = [ort.route_row(p[i], g[i], bool(cov[i]), prm, wl.prev_begin, wl.prev_count, nbr[i])
-              for i in range(N)]
+    routes = {h: [ort.route_row(p[h][i], g[i], bool(cov[i]), prm, wl.prev_begin,
+                                wl.prev_count, nbr[i]) for i in range(N)] for h in heads}
     t3 = time.perf_counter()
-    flops = 0.0
+    h0 = heads[0]
     for i in range(attn_rows):
-        tiles = routes[i][0] + routes[i][1]
-        oatt.routed_attention_block(Qh[i * b:(i + 1) * b], Kh, Vh, tiles, b)
-        flops += 4.0 * b * b * wl.d * len(tiles)
+        tiles = routes[h0][i][0] + routes[h0][i][1]
+        oatt.routed_attention_block(Qs[h0][i * b:(i + 1) * b], Ks[h0], Vh, tiles, b)
     t4 = time.perf_counter()
-    step_s = (t1 - t0) + H * (t2 - t1) + H * (t3 - t2) + (H * N / attn_rows) * (t4 - t3)
+    nh = len(heads)
+    step_s = ((t1 - t0) + (H / nh) * (t2 - t1) + (H / nh) * (t3 - t2)
+              + (H * N / attn_rows) * (t4 - t3))
+    routes = [r for h in heads for r in routes[h]]
     threads = [x.get("num_threads", 1) for x in threadpool_info()
                if x.get("user_api") == "blas"]
     mean_len = float(np.mean([len(r[0]) + len(r[1]) for r in routes]))
     return {"step_s": step_s, "sample_s": t4 - t0, "threads": max(threads) if threads else 1,
             "mean_len": mean_len,
-            "sample": (f"Gilbert neighbour table; importance of head {head} (48x2256 blocks); "
-                       f"routes of its 48 rows; attention of {attn_rows} rows; scaled to a "
-                       f"step by 40 heads and {H * N} rows")}
+            "sample": (f"Gilbert neighbour table; importance of {len(heads)} heads "
+                       f"({N}x{M} blocks each); routes of their {len(heads) * N} rows; "
+                       f"attention of {attn_rows} rows; scaled to a step of {H} heads and "
+                       f"{H * N} rows")}
 
 
 def run_reference(args, world, rank):
@@ -202,7 +205,7 @@ def run_reference(args, world, rank):
     # FLOPs of the step: mean route length of the sampled head's oracle routes
     times, flops_step = [], None
     for s in range(args.warmup + args.steps):
-        r = cpu_oracle_sample(inp, attn_rows=2)
+        r = cpu_oracle_sample(inp, attn_rows=8, heads=(0,))
         if s >= args.warmup:
             times.append(r["step_s"])
         if flops_step is None:
@@ -380,8 +383,8 @@ def _attn_source_hash() -> str:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="velox", choices=["velox", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")

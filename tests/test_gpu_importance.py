@@ -55,12 +55,12 @@ def test_importance_ragged_shapes(lib, H, N, M):
 
 
 def test_importance_peaked_logits(lib):
-    # large scale: rows nearly one-hot, still relative-accurate on the mass
+    # large scale: logits of order 100, rows nearly one-hot.  An fp32 logit
+    # carries an absolute error of about |logit| * 2^-23 ~ 1e-5, which turns
+    # into the same relative error of p: bound it at 50 * P_RTOL (1e-3).
     inp = make_inputs(small(2, 4, 50, 0, key_mean_sigma=2.0), "cuda")
     p = _run(lib, inp, 8.0)
     ref = oracle_importance(inp.Q, inp.K, range(2), 8.0)
     for h, ph in ref.items():
         g = f64(p[h])
-        big = ph > 1e-6
-        assert np.abs(g[big] / ph[big] - 1.0).max() <= 50 * P_RTOL
-        assert np.abs(g - ph).max() < 1e-6
+        assert np.all(np.abs(g - ph) <= 50 * P_RTOL * ph + 1e-30)
