@@ -125,20 +125,39 @@ def _barrier(world):
         torch.distributed.barrier()
 
 
-def _max_over_ranks(x: float, world: int) -> float:
+def _max_over_ranks(x: float, world: int, device="cuda") -> float:
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
 
-def _sum_over_ranks(x: float, world: int) -> float:
+def _sum_over_ranks(x: float, world: int, device="cuda") -> float:
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
     return float(t.item())
+
+
+def rank_workload(rank: int, heads: int = 0):
+    """Weak scaling: rank r runs layer r of the chunk-48 workload (its own
+    seeds); the path has no exchange between ranks."""
+    from synth import config
+    wl = config(3, layer=rank)
+    if heads:
+        # reduced head count: only for small profiler captures, never a bench value
+        from dataclasses import replace
+        wl = replace(wl, heads=heads)
+    return wl
+
+
+def aggregate(flops_step: float, ms_step: float, world: int, device="cuda"):
+    """Whole-job throughput: FLOPs of all ranks over the slowest rank's step."""
+    ms = _max_over_ranks(ms_step, world, device)
+    flops = _sum_over_ranks(flops_step, world, device)
+    return flops / (ms * 1e-3) / 1e12, ms
 
 
 # ---------------------------------------------------------------- oracle ---
@@ -228,10 +247,10 @@ def run_reference(args, world, rank):
 def run_velox(args, world, rank, local):
     import routed_block_sparse_b200 as rbs
     from routed_block_sparse_b200.pipeline import layer_for
-    from synth import config, make_inputs
+    from synth import make_inputs
 
     dev = torch.device("cuda", local if world > 1 else 0)
-    wl = config(3, layer=rank)  # weak scaling: each rank its own layer
+    wl = rank_workload(rank, args.heads)
     inp = make_inputs(wl, dev)
     layer = layer_for(wl, device=dev)
     H, N, M, b, d = wl.heads, wl.n_q_blocks, wl.n_kv_blocks, wl.b, wl.d
@@ -279,9 +298,7 @@ def run_velox(args, world, rank, local):
     total_ms = t_start.elapsed_time(t_end)
     parts = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])
     gil_ms, imp_ms, route_ms, attn_ms = parts.mean(axis=0)
-    ms_step = _max_over_ranks(total_ms / args.steps, world)
-    flops_all = _sum_over_ranks(flops_step, world)
-    value = flops_all / (ms_step * 1e-3) / 1e12
+    value, ms_step = aggregate(flops_step, total_ms / args.steps, world)
 
     peaks, peak_kind = _peaks()
     attn_tflops = flops_step / (attn_ms * 1e-3) / 1e12
@@ -308,7 +325,8 @@ def run_velox(args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V; g U[0,1] half zeroed; coverage Bernoulli 0.5)",
-        "config": {"workload": "chunk48", "heads": H, "n_q_blocks": N, "n_kv_blocks": M,
+        "config": {"workload": "chunk48" if H == 40 else f"chunk48 reduced to {H} heads",
+                   "heads": H, "n_q_blocks": N, "n_kv_blocks": M,
                    "head_dim": d, "b_tok": b, "k_cov": wl.params.k_cov, "k_unc": wl.params.k_unc,
                    "theta": wl.params.theta_unc, "lattice": [T, Hl, Wl],
                    "l2": "inputs larger than L2 (K+V 5.9 GB per layer), no flush"},
@@ -388,6 +406,8 @@ def main():
     ap.add_argument("--impl", default="velox", choices=["velox", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run a reduced head count (profiler captures only)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -55,7 +55,7 @@ class RouteParams(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m routed_block_sparse_b200.build`")
+                          "`python routed_block_sparse_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.velox_status_string.restype = ctypes.c_char_p

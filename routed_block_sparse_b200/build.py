@@ -1,6 +1,7 @@
 """Build libvelox.so in-tree with nvcc for sm_100a.
 
-Usage: python -m routed_block_sparse_b200.build [--verbose]
+Usage: python routed_block_sparse_b200/build.py [--force] [--verbose]
+(run it by path: importing the package loads the library it builds)
 
 Compiles every csrc/*.cu into one shared library next to this file.  The
 CUDA runtime is linked statically, so the library needs only the driver at
