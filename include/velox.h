@@ -162,6 +162,37 @@ VELOX_API velox_status velox_block_importance(const velox_bf16 *Q, const velox_b
                                     float scale, float *p, void *ws,
                                     size_t ws_bytes, velox_stream_t stream);
 
+/* Size of the fixed device scratch of velox_block_importance_noalloc. */
+#define VELOX_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/*
+ * velox_block_importance_noalloc -- velox_block_importance for callers that
+ * cannot allocate device memory.
+ *
+ * The pages have no counterpart to this call: it serves users of the
+ * library, not the method.  Some callers cannot call cudaMalloc: a host
+ * framework that budgets all device memory up front and gives its plugins
+ * no allocator, or a latency-critical loop that cannot take the device-wide
+ * synchronisation of cudaMalloc / cudaFree.  This call takes no workspace and
+ * allocates nothing; the block means live in one fixed array of
+ * VELOX_NOALLOC_SCRATCH_BYTES bytes inside the library, which every GPU that
+ * loads the library holds until the process exits.
+ *
+ * Arguments, layouts, result and device errors as velox_block_importance,
+ * without ws / ws_bytes.  Limit: H * (N + M) * d * 4 bytes must fit in the
+ * array (H * (N + M) <= 131072 at d = 128); larger sizes return
+ * VELOX_ERR_WORKSPACE before any launch.  The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress, which may load
+ * the library's device code); make that first call before any stream
+ * capture.  Every call on a device shares the one array and leaves its
+ * contents behind: calls that overlap on the GPU (other streams, unordered
+ * host threads) race on it.
+ */
+VELOX_API velox_status velox_block_importance_noalloc(const velox_bf16 *Q, const velox_bf16 *K,
+                                                      int H, int N, int M, int d, int b_tok,
+                                                      float scale, float *p,
+                                                      velox_stream_t stream);
+
 /*
  * velox_route_build -- soft geometry fusion and route materialisation.
  *

@@ -33,10 +33,11 @@ HEAD_DIM = 128
 BLOCK_TOK = 128
 MAX_BLOCKS = 65536
 MAX_ROUTE = 4096
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 EXPORTS = ("velox_status_string", "velox_abi_version", "velox_gilbert_order",
            "velox_workspace_size", "velox_block_importance", "velox_route_build",
-           "velox_block_sparse_attn")
+           "velox_block_sparse_attn", "velox_block_importance_noalloc")
 
 
 class VeloxError(RuntimeError):
@@ -68,6 +69,8 @@ def _load() -> ctypes.CDLL:
     lib.velox_workspace_size.argtypes = [I, I, I, I, ctypes.POINTER(ctypes.c_size_t)]
     lib.velox_block_importance.restype = I
     lib.velox_block_importance.argtypes = [P, P, I, I, I, I, I, F, P, P, ctypes.c_size_t, P]
+    lib.velox_block_importance_noalloc.restype = I
+    lib.velox_block_importance_noalloc.argtypes = [P, P, I, I, I, I, I, F, P, P]
     lib.velox_route_build.restype = I
     lib.velox_route_build.argtypes = [P, P, P, ctypes.POINTER(RouteParams), I, I, P, P, I, P, I,
                                       I, I, I, P, P, P, I, P, ctypes.c_size_t, P, P]
@@ -127,6 +130,14 @@ def velox_block_importance(Q, K, H, N, M, d, b_tok, scale, p, ws, stream=None):
     st = _lib.velox_block_importance(_ptr(Q), _ptr(K), H, N, M, d, b_tok, float(scale), _ptr(p),
                                      _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check("velox_block_importance", st)
+
+
+def velox_block_importance_noalloc(Q, K, H, N, M, d, b_tok, scale, p, stream=None):
+    """velox_block_importance without a workspace, for callers that cannot
+    allocate device memory (the library's fixed scratch array is used)."""
+    st = _lib.velox_block_importance_noalloc(_ptr(Q), _ptr(K), H, N, M, d, b_tok, float(scale),
+                                             _ptr(p), _stream(stream))
+    _check("velox_block_importance_noalloc", st)
 
 
 def velox_route_build(p, g, covered, prm: RouteParams, prev_begin, prev_count, nbr_ids,
