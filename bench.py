@@ -35,7 +35,7 @@ sys.path.insert(0, ROOT)
 METRIC = "routed attn µs/call & TFLOP/s at chunk-48 shape; % of B200 bf16 peak"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP = 7  # order, neighbours, pool, logits, softmax, route, attention
+LAUNCHES_PER_STEP = 7  # neighbours, pool, logits, softmax, route, schedule, attention
 
 
 def _peaks():
@@ -309,6 +309,7 @@ def run_velox(args, world, rank, local):
     ir_gbs = (imp_bytes + route_bytes) / ((imp_ms + route_ms) * 1e-3) / 1e9
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    bf16_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "attn_traffic.json")
     if os.path.exists(tpath):
@@ -335,9 +336,13 @@ def run_velox(args, world, rank, local):
         "route_us": route_ms * 1e3, "gilbert_us": gil_ms * 1e3,
         "importance_route_gbs": ir_gbs, "importance_route_hbm_frac": ir_gbs / hbm,
         "routed_tiles": tiles, "mean_route_len": tiles / (H * N), "dev_status": status,
-        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": bf16,
-                     "unit": "TFLOP/s", "frac": attn_tflops / bf16, "traffic": traffic,
-                     "peak_source": f"{peak_kind} bf16 dense (burst)"},
+        # the attention kernel is timed inside a ~1 s loop of back-to-back steps
+        # that runs under the 1 kW power cap (see "clocks"), so its denominator
+        # is the measured sustained bf16 figure; the burst fraction is reported too
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": bf16_sus,
+                     "unit": "TFLOP/s", "frac": attn_tflops / bf16_sus, "traffic": traffic,
+                     "peak_source": f"{peak_kind} bf16 dense, sustained under the power cap",
+                     "frac_of_burst_peak": attn_tflops / bf16, "burst_peak": bf16},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clocks.summary(),
     }

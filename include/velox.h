@@ -74,6 +74,7 @@ typedef enum {
 #define VELOX_DEV_BAD_SAFEGUARD  0x10  /* nbr/ref id outside [0, M): ignored   */
 #define VELOX_DEV_WAIT_TIMEOUT   0x20  /* bounded mbarrier wait gave up        */
 #define VELOX_DEV_ROUTE_CAPACITY 0x40  /* route row longer than R_max: cut     */
+#define VELOX_DEV_BAD_ROW_ORDER  0x80  /* row_order entry outside [0, H*N)      */
 
 /* Supported sizes of the importance and attention calls. */
 #define VELOX_HEAD_DIM   128
@@ -98,7 +99,7 @@ typedef struct {
 /* Human-readable text of a status; never NULL. */
 VELOX_API const char *velox_status_string(velox_status s);
 
-/* ABI version of this header (major * 100 + minor). */
+/* ABI version of this header (major * 100 + minor): 101. */
 VELOX_API int velox_abi_version(void);
 
 /*
@@ -235,6 +236,21 @@ VELOX_API velox_status velox_route_build(const float *p, const float *g,
                                int32_t *dev_status, velox_stream_t stream);
 
 /*
+ * velox_route_schedule -- the order in which velox_block_sparse_attn should
+ * take its rows: longest route first (ties keep ascending row order).
+ *
+ * The pages have no counterpart to this call: it is a launch-order hint for
+ * the attention kernel (long rows first, so the last wave of CTAs is made of
+ * short rows).  It changes no result.
+ *
+ * route_len [rows] int32 (values outside [0, R_max] count as 0), row_order
+ * [rows] int32 out: a permutation of 0 .. rows-1.  0 < R_max <=
+ * VELOX_MAX_ROUTE.
+ */
+VELOX_API velox_status velox_route_schedule(const int32_t *route_len, int rows, int R_max,
+                                            int32_t *row_order, velox_stream_t stream);
+
+/*
  * velox_block_sparse_attn -- attention over routed KV tiles.
  *
  * Defined by: digest, "Core method" (Eq. 15) and "Novelty"; project page,
@@ -250,20 +266,25 @@ VELOX_API velox_status velox_route_build(const float *p, const float *g,
  *
  * Q [H][N*b][d], K and V [H][M*b][d] bf16; O [H][N*b][d] bf16 out;
  * lse [H][N*b] fp32 out (nullable).  softmax_scale <= 0 means 1/sqrt(d).
+ * row_order [H*N] (nullable): the (h*N + i) rows in the order the CTAs take
+ * them, e.g. from velox_route_schedule; it must be a permutation of
+ * 0 .. H*N-1 (an entry outside that range is skipped and flags
+ * VELOX_DEV_BAD_ROW_ORDER).  The order changes no result.
  * d == b_tok == 128, M <= VELOX_MAX_BLOCKS, R_max <= VELOX_MAX_ROUTE when
- * routed.  A route id outside [0, M) or
- * repeated within its row is skipped (VELOX_DEV_BAD_ROUTE_ID /
- * VELOX_DEV_DUP_ROUTE_ID); route_len outside [0, R_max] zeroes the row
- * (VELOX_DEV_ROUTE_LEN).  Q, K, V, O must be 16-byte aligned.
+ * routed.  A route id outside [0, M) or repeated within its row is skipped
+ * (VELOX_DEV_BAD_ROUTE_ID / VELOX_DEV_DUP_ROUTE_ID); route_len outside
+ * [0, R_max] zeroes the row (VELOX_DEV_ROUTE_LEN).  Q, K, V, O must be
+ * 16-byte aligned.
  */
 VELOX_API velox_status velox_block_sparse_attn(const velox_bf16 *Q, const velox_bf16 *K,
-                                     const velox_bf16 *V,
-                                     const int32_t *route_ids,
-                                     const int32_t *route_len, int R_max,
-                                     int H, int N, int M, int d, int b_tok,
-                                     float softmax_scale, velox_bf16 *O,
-                                     float *lse, int32_t *dev_status,
-                                     velox_stream_t stream);
+                                               const velox_bf16 *V,
+                                               const int32_t *route_ids,
+                                               const int32_t *route_len,
+                                               const int32_t *row_order, int R_max,
+                                               int H, int N, int M, int d, int b_tok,
+                                               float softmax_scale, velox_bf16 *O,
+                                               float *lse, int32_t *dev_status,
+                                               velox_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -29,6 +29,7 @@ DEV_NBR_OVERFLOW = 0x08
 DEV_BAD_SAFEGUARD = 0x10
 DEV_WAIT_TIMEOUT = 0x20
 DEV_ROUTE_CAPACITY = 0x40
+DEV_BAD_ROW_ORDER = 0x80
 HEAD_DIM = 128
 BLOCK_TOK = 128
 MAX_BLOCKS = 65536
@@ -37,7 +38,8 @@ NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 EXPORTS = ("velox_status_string", "velox_abi_version", "velox_gilbert_order",
            "velox_workspace_size", "velox_block_importance", "velox_route_build",
-           "velox_block_sparse_attn", "velox_block_importance_noalloc")
+           "velox_block_sparse_attn", "velox_block_importance_noalloc",
+           "velox_route_schedule")
 
 
 class VeloxError(RuntimeError):
@@ -74,8 +76,10 @@ def _load() -> ctypes.CDLL:
     lib.velox_route_build.restype = I
     lib.velox_route_build.argtypes = [P, P, P, ctypes.POINTER(RouteParams), I, I, P, P, I, P, I,
                                       I, I, I, P, P, P, I, P, ctypes.c_size_t, P, P]
+    lib.velox_route_schedule.restype = I
+    lib.velox_route_schedule.argtypes = [P, I, I, P, P]
     lib.velox_block_sparse_attn.restype = I
-    lib.velox_block_sparse_attn.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, P]
+    lib.velox_block_sparse_attn.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, P]
     return lib
 
 
@@ -152,10 +156,16 @@ def velox_route_build(p, g, covered, prm: RouteParams, prev_begin, prev_count, n
     _check("velox_route_build", st)
 
 
+def velox_route_schedule(route_len, rows, R_max, row_order, stream=None):
+    st = _lib.velox_route_schedule(_ptr(route_len), rows, R_max, _ptr(row_order), _stream(stream))
+    _check("velox_route_schedule", st)
+
+
 def velox_block_sparse_attn(Q, K, V, route_ids, route_len, R_max, H, N, M, d, b_tok,
-                            softmax_scale, O, lse=None, dev_status=None, stream=None):
+                            softmax_scale, O, lse=None, dev_status=None, stream=None,
+                            row_order=None):
     st = _lib.velox_block_sparse_attn(_ptr(Q), _ptr(K), _ptr(V), _ptr(route_ids),
-                                      _ptr(route_len), R_max, H, N, M, d, b_tok,
+                                      _ptr(route_len), _ptr(row_order), R_max, H, N, M, d, b_tok,
                                       float(softmax_scale), _ptr(O), _ptr(lse),
                                       _ptr(dev_status), _stream(stream))
     _check("velox_block_sparse_attn", st)

@@ -23,8 +23,11 @@ cudaError_t launch_route(const float *p, const float *g, const uint8_t *covered,
                          const int32_t *ref_ids, int n_ref, int H, int N, int M,
                          int32_t *route_ids, int32_t *route_len, int32_t *route_nbudget,
                          int R_max, void *ws, int32_t *dev_status, cudaStream_t stream);
+cudaError_t launch_schedule(const int32_t *route_len, int rows, int R_max, int32_t *row_order,
+                            cudaStream_t stream);
 cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
-                        const int32_t *route_ids, const int32_t *route_len, int R_max, int H,
+                        const int32_t *route_ids, const int32_t *route_len,
+                        const int32_t *row_order, int R_max, int H,
                         int N, int M, float softmax_scale, uint16_t *O, float *lse,
                         int32_t *dev_status, cudaStream_t stream, bool *map_failed);
 }  // namespace velox
@@ -85,7 +88,7 @@ const char *velox_status_string(velox_status s) {
   return "unknown status";
 }
 
-int velox_abi_version(void) { return 100; }
+int velox_abi_version(void) { return 101; }
 
 velox_status velox_gilbert_order(int T, int H, int W, int n_chunks, int b_tok, int q_chunk,
                                  int cache_first_block, int n_cache_blocks,
@@ -183,9 +186,20 @@ velox_status velox_route_build(const float *p, const float *g, const uint8_t *co
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
+velox_status velox_route_schedule(const int32_t *route_len, int rows, int R_max,
+                                  int32_t *row_order, velox_stream_t stream) {
+  if (!route_len || !row_order || rows <= 0 || R_max <= 0) return VELOX_ERR_INVALID_ARG;
+  if (R_max > VELOX_MAX_ROUTE) return VELOX_ERR_UNSUPPORTED;
+  velox_status st = check_device();
+  if (st != VELOX_OK) return st;
+  return from_cuda(velox::launch_schedule(route_len, rows, R_max, row_order,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
 velox_status velox_block_sparse_attn(const velox_bf16 *Q, const velox_bf16 *K,
                                      const velox_bf16 *V, const int32_t *route_ids,
-                                     const int32_t *route_len, int R_max, int H, int N, int M,
+                                     const int32_t *route_len, const int32_t *row_order,
+                                     int R_max, int H, int N, int M,
                                      int d, int b_tok, float softmax_scale, velox_bf16 *O,
                                      float *lse, int32_t *dev_status, velox_stream_t stream) {
   if (!Q || !K || !V || !O || H <= 0 || N <= 0 || M <= 0) return VELOX_ERR_INVALID_ARG;
@@ -193,6 +207,7 @@ velox_status velox_block_sparse_attn(const velox_bf16 *Q, const velox_bf16 *K,
   if (M > VELOX_MAX_BLOCKS || (long long)M * b_tok > kInt32Max ||
       (long long)N * b_tok > kInt32Max || (long long)H * N > kInt32Max)
     return VELOX_ERR_UNSUPPORTED;
+  if (row_order != nullptr && dev_status == nullptr) return VELOX_ERR_INVALID_ARG;
   if (route_ids != nullptr) {
     if (route_len == nullptr || dev_status == nullptr) return VELOX_ERR_INVALID_ARG;
     if (R_max <= 0) return VELOX_ERR_INVALID_ARG;
@@ -205,7 +220,8 @@ velox_status velox_block_sparse_attn(const velox_bf16 *Q, const velox_bf16 *K,
   velox_status st = check_device();
   if (st != VELOX_OK) return st;
   bool map_failed = false;
-  cudaError_t e = velox::launch_attn(Q, K, V, route_ids, route_len, R_max, H, N, M, scale, O, lse,
+  cudaError_t e = velox::launch_attn(Q, K, V, route_ids, route_len, row_order, R_max, H, N, M,
+                                     scale, O, lse,
                                      dev_status, reinterpret_cast<cudaStream_t>(stream),
                                      &map_failed);
   if (map_failed) return VELOX_ERR_CUDA;

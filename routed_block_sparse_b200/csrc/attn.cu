@@ -7,23 +7,27 @@
 // attention restricted to the tokens of the listed tiles, computed with the
 // FlashAttention online-softmax recurrence over tiles.
 //
-// sm_100a design: one CTA per (head, query block), two CTAs per SM.  Within a
-// CTA the chain S_j -> softmax_j -> PV_j is serial (P lives in the TMEM
-// columns of S), and the second CTA on the SM fills the tensor core while the
-// first one runs its softmax, so the two query blocks ping-pong on the SM.
-//   warp 0      TMA producer: Q once, then the K and V tiles of the route
-//               (128-byte swizzle, two 64-channel boxes per tile); K_{j+1} is
-//               fetched as soon as S_j is done, V_{j+1} as soon as PV_j is.
-//   warp 1      TMEM allocator (256 columns: S/P 128, O 128) and the single
-//               tcgen05.mma issuer: S_j = Q K_j^T (A, B from shared memory),
-//               O += P_j V_j (A = P from TMEM, B = V from shared memory).
-//   warps 2-5   softmax: one query row per thread (its TMEM lane).  Row max
-//               with independent partial maxima, exponentials in the log2
-//               domain, P_j packed to bf16 into the S columns with
-//               tcgen05.st.  The running max is only moved (and O rescaled in
-//               TMEM) when it grows by more than 2^8; otherwise the stale max
-//               is kept, which is exact because O and the row sum always use
-//               the same max.  Epilogue: O / l -> bf16, lse.
+// sm_100a design: one CTA per (head, query block), one CTA per SM, all 512
+// TMEM columns: three S buffers (128 columns each) and the O accumulator.
+// CTAs take rows in the order `row_order` gives (longest routes first, from
+// velox_route_schedule), so the last wave is made of short rows.
+//   warp 0      TMA producer: Q once, then K_0, V_0, K_1, V_1, ... of the
+//               route into a ring of 32 KB slots (128-byte swizzle, two
+//               64-channel boxes per tile).
+//   warp 1      TMEM allocator and the single tcgen05.mma issuer.  It keeps
+//               the score products two tiles ahead of the softmax: as soon as
+//               PV_{j-1} has completed it issues S_{j+2} = Q K_{j+2}^T into the
+//               buffer P_{j-1} occupied, then O += P_j V_j (A = P from TMEM,
+//               B = V from shared memory) once the softmax of tile j is done.
+//   warps 2-5   softmax: one query row per thread (its TMEM lane).  One
+//               TMEM read of the S row, row max with three-input max, scaled
+//               exponent arguments and the row sum in packed fp32x2
+//               arithmetic, exponentials on MUFU, P_j packed to bf16 into the
+//               first 64 columns of its own S buffer.  The running max is
+//               only moved (and O rescaled in TMEM, after waiting for
+//               PV_{j-1}) when it grows by more than 2^8; otherwise the stale
+//               max is kept, which is exact because O and the row sum always
+//               use the same max.  Epilogue: O / l -> bf16, lse.
 // A pre-pass compacts the route into shared memory, skipping ids outside
 // [0, M) and repeats (flagged in dev_status).
 #include <cudaTypedefs.h>
@@ -42,30 +46,35 @@ constexpr int kThreads = 192;
 constexpr uint32_t kTileBytes = BN * D * 2;      // 32 KB
 constexpr uint32_t kHalfBytes = kTileBytes / 2;  // one 64-channel box
 constexpr int kMaxRoute = VELOX_MAX_ROUTE;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0;    // S (fp32, 128 columns); P (bf16x2) in its first 64
-constexpr uint32_t kColO = 128;  // O accumulator (fp32, 128 columns)
+constexpr uint32_t kTmemCols = 512;
+constexpr int kSBufs = 3;         // S/P buffers in TMEM, columns 0, 128, 256
+constexpr uint32_t kColO = 384;   // O accumulator (fp32, 128 columns)
+constexpr int kMaxSlots = 6;      // K/V ring slots of 32 KB
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest tolerated growth
 
 // shared-memory layout (offsets from a 1024-byte aligned base)
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTileBytes;
-constexpr uint32_t kOffV = kOffK + kTileBytes;
-constexpr uint32_t kOffBar = kOffV + kTileBytes;
-constexpr uint32_t kNumBars = 10;
-constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-constexpr uint32_t kOffDyn = kOffMisc + 64;  // route list (uint16), then the id bitmap
+constexpr uint32_t kOffRing = kOffQ + kTileBytes;
+// barriers, misc and the dynamic tail follow the ring (offset set at launch)
+constexpr uint32_t kNumBars = 1 + 2 * kMaxSlots + 3 * kSBufs + 1;
+constexpr uint32_t kMiscBytes = 64;
+constexpr uint32_t kSmemLimit = 227 * 1024;
 
 struct AttnArgs {
   const int32_t *route_ids;  // null: dense
   const int32_t *route_len;
+  const int32_t *row_order;  // null: row = blockIdx.x
   int R_max;
   int N, M;
+  int rows;                  // H * N
   float scale_log2;  // softmax_scale * log2(e)
   uint16_t *O;
   float *lse;
   int32_t *dev_status;
-  uint32_t bits_offset;  // byte offset of the id bitmap from the aligned base
+  int nslot;              // K/V ring slots in use (4..kMaxSlots)
+  uint32_t bar_offset;    // byte offset of the barriers from the aligned base
+  uint32_t list_offset;   // route list (uint16)
+  uint32_t bits_offset;   // id bitmap (uint32)
 };
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_saddr, int k) {
@@ -95,41 +104,52 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
   uint8_t *sQ = base + kOffQ;
-  uint8_t *sK = base + kOffK;
-  uint8_t *sV = base + kOffV;
-  uint64_t *bar = reinterpret_cast<uint64_t *>(base + kOffBar);
-  uint64_t *q_full = bar + 0, *k_full = bar + 1, *k_empty = bar + 2, *v_full = bar + 3,
-           *v_empty = bar + 4, *s_full = bar + 5, *p_full = bar + 6, *o_done = bar + 7,
-           *mma_done = bar + 8;
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(base + kOffMisc);
-  int *s_nvalid = reinterpret_cast<int *>(base + kOffMisc + 4);
-  volatile int *s_abort = reinterpret_cast<volatile int *>(base + kOffMisc + 8);
-  uint16_t *tiles = reinterpret_cast<uint16_t *>(base + kOffDyn);
+  uint8_t *ring = base + kOffRing;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(base + a.bar_offset);
+  uint64_t *q_full = bar;
+  uint64_t *slot_full = bar + 1;
+  uint64_t *slot_empty = slot_full + kMaxSlots;
+  uint64_t *s_full = slot_empty + kMaxSlots;
+  uint64_t *p_full = s_full + kSBufs;
+  uint64_t *pv_done = p_full + kSBufs;
+  uint64_t *mma_done = pv_done + kSBufs;
+  uint8_t *misc = base + a.bar_offset + kNumBars * 8;
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(misc);
+  int *s_nvalid = reinterpret_cast<int *>(misc + 4);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(misc + 8);
+  uint16_t *tiles = reinterpret_cast<uint16_t *>(base + a.list_offset);
   uint32_t *bits = reinterpret_cast<uint32_t *>(base + a.bits_offset);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x;
+  const int row = a.row_order ? a.row_order[blockIdx.x] : (int)blockIdx.x;
+  if (row < 0 || row >= a.rows) {  // same value in every thread: uniform exit
+    if (threadIdx.x == 0) flag_error(a.dev_status, VELOX_DEV_BAD_ROW_ORDER);
+    return;
+  }
   const int h = row / a.N, i = row - h * a.N;
   const bool dense = (a.route_ids == nullptr);
   const int M = a.M;
+  const int nslot = a.nslot;
 
   // ---- set-up: barriers, TMEM, route compaction
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    mbar_init(k_full, 1);
-    mbar_init(k_empty, 1);
-    mbar_init(v_full, 1);
-    mbar_init(v_empty, 1);
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
+    for (int s = 0; s < kMaxSlots; ++s) {
+      mbar_init(&slot_full[s], 1);
+      mbar_init(&slot_empty[s], 1);
+    }
+    for (int b = 0; b < kSBufs; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 128);
+      mbar_init(&pv_done[b], 1);
+    }
     mbar_init(mma_done, 1);
     *s_abort = 0;
     fence_mbar_init();
@@ -192,33 +212,28 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_arrive_expect_tx(q_full, kTileBytes);
       tma_load_3d(sQ, &tmQ, q_full, 0, i * BM, h);
       tma_load_3d(sQ + kHalfBytes, &tmQ, q_full, 64, i * BM, h);
-      int k_issued = 0, v_issued = 0;
-      for (int j = 0; j < n; ++j) {
-        const uint32_t free_parity = (j & 1) ^ 1;
+      int issued = 0;
+      for (int li = 0; li < 2 * n; ++li) {  // load li: K_{li/2} (even) or V_{li/2} (odd)
+        const int s = li % nslot;
+        const uint32_t use = li / nslot;
+        if (!mbar_wait(&slot_empty[s], (use & 1) ^ 1, s_abort)) break;
+        const int j = li >> 1;
         const int tile = dense ? j : tiles[j];
-        if (!mbar_wait(k_empty, free_parity, s_abort)) break;
-        mbar_arrive_expect_tx(k_full, kTileBytes);
-        tma_load_3d(sK, &tmK, k_full, 0, tile * BN, h);
-        tma_load_3d(sK + kHalfBytes, &tmK, k_full, 64, tile * BN, h);
-        k_issued = j + 1;
-        if (!mbar_wait(v_empty, free_parity, s_abort)) break;
-        mbar_arrive_expect_tx(v_full, kTileBytes);
-        tma_load_3d(sV, &tmV, v_full, 0, tile * BN, h);
-        tma_load_3d(sV + kHalfBytes, &tmV, v_full, 64, tile * BN, h);
-        v_issued = j + 1;
+        const CUtensorMap *map = (li & 1) ? &tmV : &tmK;
+        uint8_t *dst = ring + s * kTileBytes;
+        mbar_arrive_expect_tx(&slot_full[s], kTileBytes);
+        tma_load_3d(dst, map, &slot_full[s], 0, tile * BN, h);
+        tma_load_3d(dst + kHalfBytes, map, &slot_full[s], 64, tile * BN, h);
+        issued = li + 1;
       }
       if (*s_abort) {
         // let the copies already in flight land before the CTA goes away
         // (each wait is bounded by the same time limit)
         volatile int never = 0;
         mbar_wait(q_full, 0, &never);
-        if (k_issued > 0) {
+        for (int li = issued - nslot < 0 ? 0 : issued - nslot; li < issued; ++li) {
           never = 0;
-          mbar_wait(k_full, (k_issued - 1) & 1, &never);
-        }
-        if (v_issued > 0) {
-          never = 0;
-          mbar_wait(v_full, (v_issued - 1) & 1, &never);
+          mbar_wait(&slot_full[li % nslot], (li / nslot) & 1, &never);
         }
       }
     }
@@ -227,28 +242,44 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0 && n > 0) {
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false);
       constexpr uint32_t idPV = idesc_bf16_f32(BM, D, true);
-      const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV);
-      bool ok = mbar_wait(q_full, 0, s_abort);
-      for (int j = 0; ok && j < n; ++j) {
-        const uint32_t ph = j & 1;
-        if (!mbar_wait(k_full, ph, s_abort)) break;
-        // S_j overwrites the columns P_{j-1} was read from
-        if (j > 0 && !mbar_wait(o_done, ph ^ 1, s_abort)) break;
+      const uint32_t qa = smem_u32(sQ), ra = smem_u32(ring);
+      auto issue_s = [&](int j) -> bool {
+        const int li = 2 * j, s = li % nslot;
+        if (!mbar_wait(&slot_full[s], (li / nslot) & 1, s_abort)) return false;
         tc_fence_after();
+        const uint32_t ka = ra + s * kTileBytes;
+        const uint32_t sb = tmem + (j % kSBufs) * BN;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_bf16_ss(tmem + kColS, kmajor_desc(qa, k), kmajor_desc(ka, k), idS, k > 0);
-        tc_commit(s_full);
-        tc_commit(k_empty);
-        if (!mbar_wait(p_full, ph, s_abort)) break;
-        if (!mbar_wait(v_full, ph, s_abort)) break;
+          mma_bf16_ss(sb, kmajor_desc(qa, k), kmajor_desc(ka, k), idS, k > 0);
+        tc_commit(&s_full[j % kSBufs]);
+        tc_commit(&slot_empty[s]);
+        return true;
+      };
+      bool ok = mbar_wait(q_full, 0, s_abort);
+      if (ok) ok = issue_s(0);
+      if (ok && n > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < n; ++j) {
+        const int b = j % kSBufs;
+        if (j + 2 < n) {
+          // S_{j+2} goes into the buffer P_{j-1} occupied: PV_{j-1} must be done
+          if (j >= 1) {
+            const int jp = j - 1;
+            if (!mbar_wait(&pv_done[jp % kSBufs], (jp / kSBufs) & 1, s_abort)) break;
+          }
+          if (!issue_s(j + 2)) break;
+        }
+        if (!mbar_wait(&p_full[b], (j / kSBufs) & 1, s_abort)) break;
+        const int li = 2 * j + 1, s = li % nslot;
+        if (!mbar_wait(&slot_full[s], (li / nslot) & 1, s_abort)) break;
         tc_fence_after();
+        const uint32_t va = ra + s * kTileBytes;
+        const uint32_t pb = tmem + b * BN;  // P_j: first 64 columns of its S buffer
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k)
-          mma_bf16_ts(tmem + kColO, tmem + kColS + k * 8, vmn_desc(va, k), idPV,
-                      (j > 0 || k > 0));
-        tc_commit(o_done);
-        tc_commit(v_empty);
+          mma_bf16_ts(tmem + kColO, pb + k * 8, vmn_desc(va, k), idPV, (j > 0 || k > 0));
+        tc_commit(&pv_done[b]);
+        tc_commit(&slot_empty[s]);
       }
       // all issued MMAs must be complete before TMEM is released
       tc_commit(mma_done);
@@ -264,82 +295,80 @@ __global__ void __launch_bounds__(kThreads, 2)
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
-      const uint32_t ph = j & 1;
-      if (!warp_wait(s_full, ph, s_abort)) { ok = false; break; }
+      const int b = j % kSBufs;
+      const uint32_t sb = trow + b * BN;
+      if (!warp_wait(&s_full[b], (j / kSBufs) & 1, s_abort)) { ok = false; break; }
       tc_fence_after();
-      // pass 1: row max (independent partial maxima)
+      uint32_t sv[128];
+      tmem_ld32(sb, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(sb + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_ld32(sb + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+      tmem_ld32(sb + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+      tmem_wait_ld();
       float mx[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t s0[32], s1[32];
-        tmem_ld32(trow + kColS + half * 64, s0);
-        tmem_ld32(trow + kColS + half * 64 + 32, s1);
-        tmem_wait_ld();
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          mx[k & 7] = fmaxf(mx[k & 7], __uint_as_float(s0[k]));
-          mx[k & 7] = fmaxf(mx[k & 7], __uint_as_float(s1[k]));
-        }
-      }
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      for (int k = 0; k < 64; ++k)
+        mx[k & 7] = fmax3(mx[k & 7], __uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1]));
+      const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                             fmaxf(mx[6], mx[7]));
       const float m_cand = fmaxf(m_run, mt * c);
       const bool grow = m_cand > m_run + kRescaleThreshold;  // always on the first tile
       const float m_use = grow ? m_cand : m_run;
       const float alpha = fast_exp2(m_run - m_use);  // 1 if kept, 0 on the first tile
-      // pass 2: exponentials, row sum, bf16 packing.  s_full(j) implies that
-      // PV_{j-1} is complete (the MMA warp waited for it before issuing S_j),
-      // so P_j may go into the S columns already read: column t/2 holds
-      // elements t, t+1 (lower index in the low half).
-      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // move O to the new max: PV_{j-1} (and every earlier PV) must be done
+        const int jp = j - 1;
+        if (!warp_wait(&pv_done[jp % kSBufs], (jp / kSBufs) & 1, s_abort)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t ov[32];
+          tmem_ld32(trow + kColO + cc * 32, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
+          tmem_st32(trow + kColO + cc * 32, ov);
+        }
+      }
+      // exponentials (arguments and row sum in packed pairs); P_j into the
+      // first 64 columns of its S buffer: column t/2 holds elements t, t+1
+      uint64_t sum2[2] = {0ull, 0ull};
+      const uint64_t c2 = f2pack(c, c), nm2 = f2pack(-m_use, -m_use);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        uint32_t s0[32], s1[32];
-        tmem_ld32(trow + kColS + half * 64, s0);
-        tmem_ld32(trow + kColS + half * 64 + 32, s1);
-        tmem_wait_ld();
         uint32_t pk[32];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(s0[2 * k]), c, -m_use));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(s0[2 * k + 1]), c, -m_use));
-          const float p2 = fast_exp2(fmaf(__uint_as_float(s1[2 * k]), c, -m_use));
-          const float p3 = fast_exp2(fmaf(__uint_as_float(s1[2 * k + 1]), c, -m_use));
-          sum[k & 3] += (p0 + p1) + (p2 + p3);
+        for (int k = 0; k < 32; ++k) {
+          const uint64_t x2 = ffma2(f2pack(__uint_as_float(sv[half * 64 + 2 * k]),
+                                           __uint_as_float(sv[half * 64 + 2 * k + 1])),
+                                    c2, nm2);
+          float x0, x1;
+          f2unpack(x2, x0, x1);
+          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          sum2[k & 1] = fadd2(sum2[k & 1], f2pack(p0, p1));
           pk[k] = pack_bf16x2(p0, p1);
-          pk[16 + k] = pack_bf16x2(p2, p3);
         }
-        tmem_st32(trow + kColS + half * 32, pk);
+        tmem_st32(sb + half * 32, pk);
       }
-      if (j > 0) {
-        // O is stable (PV_{j-1} done); move it to the new max when any row of
-        // the warp grew past the threshold
-        if (!warp_wait(o_done, ph ^ 1, s_abort)) { ok = false; break; }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t ov[32];
-            tmem_ld32(trow + kColO + cc * 32, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
-            tmem_st32(trow + kColO + cc * 32, ov);
-          }
-        }
-      }
+      float sa, sb2, sc, sd;
+      f2unpack(fadd2(sum2[0], sum2[1]), sa, sb2);
       tmem_wait_st();
-      l = l * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
+      l = l * alpha + (sa + sb2);
       m_run = m_use;
+      (void)sc;
+      (void)sd;
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[b]);
     }
     // epilogue
     uint16_t *orow = a.O + ((size_t)row * BM + r) * D;
     bool have = ok && n > 0;
-    if (have) have = mbar_wait(o_done, (n - 1) & 1, s_abort);
+    if (have) {
+      const int jl = n - 1;
+      have = mbar_wait(&pv_done[jl % kSBufs], (jl / kSBufs) & 1, s_abort);
+    }
     // tcgen05.ld is warp-collective: decide once for the whole warp
     const bool good = __all_sync(0xffffffffu, have && !*s_abort);
     tc_fence_after();
@@ -410,7 +439,8 @@ bool make_map(CUtensorMap *map, const void *ptr, int rows, int H) {
 int attn_max_route() { return kMaxRoute; }
 
 cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
-                        const int32_t *route_ids, const int32_t *route_len, int R_max, int H,
+                        const int32_t *route_ids, const int32_t *route_len,
+                        const int32_t *row_order, int R_max, int H,
                         int N, int M, float softmax_scale, uint16_t *O, float *lse,
                         int32_t *dev_status, cudaStream_t stream, bool *map_failed) {
   *map_failed = false;
@@ -423,18 +453,27 @@ cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
   AttnArgs a;
   a.route_ids = route_ids;
   a.route_len = route_len;
+  a.row_order = row_order;
   a.R_max = R_max;
   a.N = N;
   a.M = M;
+  a.rows = H * N;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.O = O;
   a.lse = lse;
   a.dev_status = dev_status;
-  // dynamic tail: route list (uint16 x R_max, 16-byte rounded), id bitmap
-  uint32_t list_bytes = route_ids ? ((uint32_t)R_max * 2u + 15u) & ~15u : 0u;
-  uint32_t bits_bytes = route_ids ? (uint32_t)((M + 31) / 32) * 4u : 0u;
-  a.bits_offset = kOffDyn + list_bytes;
+  // tail after the ring: barriers, misc, route list (uint16), id bitmap
+  const uint32_t list_bytes = route_ids ? ((uint32_t)R_max * 2u + 15u) & ~15u : 0u;
+  const uint32_t bits_bytes = route_ids ? (uint32_t)((M + 31) / 32) * 4u : 0u;
+  const uint32_t tail = kNumBars * 8 + kMiscBytes + list_bytes + bits_bytes;
+  int nslot = kMaxSlots;
+  while (nslot > 4 && kOffRing + nslot * kTileBytes + tail + 1024 > kSmemLimit) --nslot;
+  a.nslot = nslot;
+  a.bar_offset = kOffRing + nslot * kTileBytes;
+  a.list_offset = a.bar_offset + kNumBars * 8 + kMiscBytes;
+  a.bits_offset = a.list_offset + list_bytes;
   const size_t smem = (size_t)a.bits_offset + bits_bytes + 1024;  // + alignment slack
+  if (smem > kSmemLimit) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;

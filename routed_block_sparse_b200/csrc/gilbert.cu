@@ -133,64 +133,76 @@ __global__ void order_kernel(Lattice L, int n_cells, int32_t *rank_of_cell,
   }
 }
 
-// One CTA per query block of chunk q_chunk.  Candidates (26 offsets of each
-// of the b tokens) are gathered in shared memory, sorted, deduplicated.
+// One CTA per query block i of chunk q_chunk.  The neighbours of a block
+// whose tokens span global frames f0..f1 lie in frames f0-1 .. f1+1, hence in
+// a window of block ids [wlo, whi]; a bitmap over that window collects them
+// without repeats, and a scan of the bitmap writes them in ascending order.
+// When a frame has at most kFrameSmemCells cells, the frame's rank map and its
+// inverse are built once in shared memory and every lookup is a table read;
+// otherwise each lookup descends the recursion.
+constexpr int kFrameSmemCells = 8192;
+
 __global__ void neighbour_kernel(Lattice L, int q_chunk, int cache_first, int n_cache,
-                                 int32_t *nbr_ids, int32_t *nbr_cnt, int S_max, int cap,
+                                 int32_t *nbr_ids, int32_t *nbr_cnt, int S_max, int use_table,
                                  int32_t *dev_status) {
-  extern __shared__ int cand[];  // cap entries (a power of two)
-  __shared__ int s_count;
-  __shared__ int s_scan[1024];
-  const int per_chunk = L.T * L.H * L.W / L.b;
+  extern __shared__ int smem_i[];
+  __shared__ int s_scan[256];
+  const int HW = L.HW();
+  int *r2 = smem_i;                             // [HW] when use_table
+  int *inv = smem_i + (use_table ? HW : 0);     // [HW] when use_table
+  uint32_t *win = reinterpret_cast<uint32_t *>(smem_i + (use_table ? 2 * HW : 0));
+  const int per_chunk = L.T * HW / L.b;
   const int i = blockIdx.x;
   const int qb = q_chunk * per_chunk + i;
-  for (int k = threadIdx.x; k < cap; k += blockDim.x) cand[k] = INT32_MAX;
-  if (threadIdx.x == 0) s_count = 0;
-  __syncthreads();
-  const int HW = L.HW();
   const int F = L.n_chunks * L.T;
-  for (int t = threadIdx.x; t < L.b; t += blockDim.x) {
-    int rank = qb * L.b + t;
-    int f = rank / HW;
-    int k = rank - f * HW;
-    int xm, y;
-    frame_cell(L.W, L.H, k, xm, y);
-    int x = (f & 1) ? (L.W - 1 - xm) : xm;
-    for (int o = 0; o < 27; ++o) {
-      if (o == 13) continue;  // the centre
-      int f2 = f + o / 9 - 1, y2 = y + (o / 3) % 3 - 1, x2 = x + o % 3 - 1;
-      if (f2 < 0 || f2 >= F || y2 < 0 || y2 >= L.H || x2 < 0 || x2 >= L.W) continue;
-      int u = L.rank(f2, y2, x2) / L.b;
-      if (u == qb || u < cache_first || u >= cache_first + n_cache) continue;
-      int slot = atomicAdd(&s_count, 1);
-      cand[slot] = u - cache_first;  // slot < 26 * b <= cap by construction
+  const long long first_rank = (long long)qb * L.b;
+  const int f0 = (int)(first_rank / HW), f1 = (int)((first_rank + L.b - 1) / HW);
+  const int wf0 = f0 > 0 ? f0 - 1 : 0, wf1 = f1 + 1 < F ? f1 + 1 : F - 1;
+  const int wlo = (int)((long long)wf0 * HW / L.b);
+  const int whi = (int)(((long long)(wf1 + 1) * HW - 1) / L.b);
+  const int nwin = whi - wlo + 1;
+  const int nwords = (nwin + 31) >> 5;
+  for (int k = threadIdx.x; k < nwords; k += blockDim.x) win[k] = 0u;
+  if (use_table) {
+    for (int cidx = threadIdx.x; cidx < HW; cidx += blockDim.x) {
+      const int y = cidx / L.W, x = cidx - y * L.W;
+      const int rk = frame_rank(L.W, L.H, x, y);
+      r2[cidx] = rk;
+      inv[rk] = cidx;
     }
   }
   __syncthreads();
-  // bitonic sort of cap entries (INT32_MAX padding sorts last)
-  for (int size = 2; size <= cap; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int k = threadIdx.x; k < cap; k += blockDim.x) {
-        int partner = k ^ stride;
-        if (partner > k) {
-          bool up = ((k & size) == 0);
-          int a = cand[k], b2 = cand[partner];
-          if ((a > b2) == up) {
-            cand[k] = b2;
-            cand[partner] = a;
-          }
-        }
-      }
-      __syncthreads();
+  const int items = L.b * 26;
+  for (int it = threadIdx.x; it < items; it += blockDim.x) {
+    const int t = it / 26, o26 = it - t * 26;
+    const int o = o26 < 13 ? o26 : o26 + 1;  // skip the centre offset 13
+    const long long rank = first_rank + t;
+    const int f = (int)(rank / HW);
+    const int k = (int)(rank - (long long)f * HW);
+    int xm, y;
+    if (use_table) {
+      const int cidx = inv[k];
+      y = cidx / L.W;
+      xm = cidx - y * L.W;
+    } else {
+      frame_cell(L.W, L.H, k, xm, y);
     }
+    const int x = (f & 1) ? (L.W - 1 - xm) : xm;
+    const int f2 = f + o / 9 - 1, y2 = y + (o / 3) % 3 - 1, x2 = x + o % 3 - 1;
+    if (f2 < 0 || f2 >= F || y2 < 0 || y2 >= L.H || x2 < 0 || x2 >= L.W) continue;
+    const int xm2 = (f2 & 1) ? (L.W - 1 - x2) : x2;
+    const int r2v = use_table ? r2[y2 * L.W + xm2] : frame_rank(L.W, L.H, xm2, y2);
+    const int u = (int)(((long long)f2 * HW + r2v) / L.b);
+    if (u == qb || u < cache_first || u >= cache_first + n_cache) continue;
+    const int bit = u - wlo;  // within the window by construction
+    atomicOr(&win[bit >> 5], 1u << (bit & 31));
   }
-  // keep the first of each run of equal ids: ordered compaction, thread t
-  // owning a contiguous chunk of the sorted array
-  const int n = s_count;
-  const int chunk = (n + blockDim.x - 1) / blockDim.x;
-  const int lo = threadIdx.x * chunk, hi = min(n, lo + chunk);
+  __syncthreads();
+  // ordered write-out: thread t owns a contiguous run of bitmap words
+  const int wchunk = (nwords + blockDim.x - 1) / blockDim.x;
+  const int wl = min(nwords, (int)threadIdx.x * wchunk), wh = min(nwords, wl + wchunk);
   int mine = 0;
-  for (int k = lo; k < hi; ++k) mine += (k == 0 || cand[k] != cand[k - 1]);
+  for (int k = wl; k < wh; ++k) mine += __popc(win[k]);
   s_scan[threadIdx.x] = mine;
   __syncthreads();
   for (int off = 1; off < (int)blockDim.x; off <<= 1) {
@@ -201,9 +213,12 @@ __global__ void neighbour_kernel(Lattice L, int q_chunk, int cache_first, int n_
   }
   const int total = s_scan[blockDim.x - 1];
   int pos = s_scan[threadIdx.x] - mine;
-  for (int k = lo; k < hi; ++k) {
-    if (k == 0 || cand[k] != cand[k - 1]) {
-      if (pos < S_max && nbr_ids) nbr_ids[(size_t)i * S_max + pos] = cand[k];
+  for (int k = wl; k < wh; ++k) {
+    uint32_t w = win[k];
+    while (w) {
+      const int bit = __ffs(w) - 1;
+      w &= w - 1;
+      if (pos < S_max && nbr_ids) nbr_ids[(size_t)i * S_max + pos] = wlo + (k << 5) + bit - cache_first;
       ++pos;
     }
   }
@@ -233,10 +248,15 @@ cudaError_t launch_gilbert(int T, int H, int W, int n_chunks, int b, int q_chunk
     if (e != cudaSuccess) return e;
   }
   if (nbr_ids || nbr_cnt) {
-    int cap = 1;
-    while (cap < 26 * b) cap <<= 1;
-    const int per_chunk = T * H * W / b;
-    size_t smem = (size_t)cap * sizeof(int);
+    const int HW = H * W;
+    const int per_chunk = T * HW / b;
+    const int use_table = HW <= kFrameSmemCells ? 1 : 0;
+    // window of candidate block ids: at most (frames spanned + 2) frames
+    const long long span_frames = (b + HW - 1) / HW + 1;
+    const long long nwin = ((span_frames + 2) * HW) / b + 2;
+    size_t smem = (use_table ? (size_t)2 * HW * sizeof(int) : 0) +
+                  (size_t)((nwin + 31) / 32) * sizeof(uint32_t);
+    if (smem > 200 * 1024) return cudaErrorInvalidValue;
     if (smem > 48 * 1024) {
       cudaError_t e = cudaFuncSetAttribute(neighbour_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -244,7 +264,7 @@ cudaError_t launch_gilbert(int T, int H, int W, int n_chunks, int b, int q_chunk
       if (e != cudaSuccess) return e;
     }
     neighbour_kernel<<<per_chunk, 256, smem, stream>>>(L, q_chunk, cache_first, n_cache,
-                                                       nbr_ids, nbr_cnt, S_max, cap,
+                                                       nbr_ids, nbr_cnt, S_max, use_table,
                                                        dev_status);
     return cudaGetLastError();
   }

@@ -7,6 +7,9 @@ C entry points; the arithmetic of every step runs in libvelox.so.
                         prev_count=48, lattice=(4, 32, 48), q_chunk=47)
     O, lse = layer.forward(Q, K, V, g, covered)
 
+The route build is followed by velox_route_schedule (longest routes first), whose
+order the attention launch follows.
+
 Step order (Velox project page, "02 · Method", steps 03-04; digest of arXiv
 2610.22311, "Method steps", step four and five): block importance -> soft
 fusion and route -> block-sparse attention.  The Gilbert neighbour table is
@@ -21,7 +24,7 @@ import torch
 
 from . import (BLOCK_TOK, HEAD_DIM, RouteParams, route_params, velox_block_importance,
                velox_block_sparse_attn, velox_gilbert_order, velox_route_build,
-               velox_workspace_size)
+               velox_route_schedule, velox_workspace_size)
 
 DEFAULT_S_MAX = 64
 
@@ -64,6 +67,7 @@ class RoutedLayer:
         self.route_ids = torch.empty(H, N, self.R_max, dtype=i32, device=dev)
         self.route_len = torch.empty(H, N, dtype=i32, device=dev)
         self.route_nbudget = torch.empty(H, N, dtype=i32, device=dev)
+        self.row_order = torch.empty(H * N, dtype=i32, device=dev)
         self.O = torch.empty(H, N * self.b, self.d, dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty(H, N * self.b, dtype=torch.float32, device=dev)
 
@@ -79,13 +83,15 @@ class RoutedLayer:
                           self.ref_ids, self.n_ref, self.H, self.N, self.M, self.route_ids,
                           self.route_len, self.route_nbudget, self.R_max, self.ws,
                           self.dev_status, stream)
+        velox_route_schedule(self.route_len, self.H * self.N, self.R_max, self.row_order, stream)
         return self.route_ids, self.route_len, self.route_nbudget
 
     def attend(self, Q, K, V, dense: bool = False, stream=None):
         velox_block_sparse_attn(Q, K, V, None if dense else self.route_ids,
                                 None if dense else self.route_len, self.R_max, self.H, self.N,
                                 self.M, self.d, self.b, self.softmax_scale, self.O, self.lse,
-                                self.dev_status, stream)
+                                self.dev_status, stream,
+                                row_order=None if dense else self.row_order)
         return self.O, self.lse
 
     def forward(self, Q, K, V, g, covered, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:

@@ -60,7 +60,7 @@ def test_binding_names_match_header(built):
 
 def test_status_strings_and_version(built):
     import routed_block_sparse_b200 as rbs
-    assert rbs.velox_abi_version() == 100
+    assert rbs.velox_abi_version() == 101
     for s in range(8):
         assert isinstance(rbs.velox_status_string(s), str) and rbs.velox_status_string(s)
     assert rbs.velox_status_string(99) == "unknown status"
@@ -81,21 +81,28 @@ def test_invalid_arguments_rejected_before_any_launch(built):
     lib.velox_block_sparse_attn.restype = ctypes.c_int
     P = ctypes.c_void_p
     # null pointers -> VELOX_ERR_INVALID_ARG (1)
-    st = lib.velox_block_sparse_attn(None, None, None, None, None, 0, 1, 1, 1, 128, 128,
+    st = lib.velox_block_sparse_attn(None, None, None, None, None, None, 0, 1, 1, 1, 128, 128,
                                      ctypes.c_float(0.0), None, None, None, None)
     assert st == 1
     fake = P(0x10000)
     # unsupported head dim -> VELOX_ERR_UNSUPPORTED (2)
-    st = lib.velox_block_sparse_attn(fake, fake, fake, None, None, 0, 1, 1, 1, 64, 128,
+    st = lib.velox_block_sparse_attn(fake, fake, fake, None, None, None, 0, 1, 1, 1, 64, 128,
                                      ctypes.c_float(0.0), fake, None, None, None)
     assert st == 2
     # R_max above the routed limit -> unsupported
-    st = lib.velox_block_sparse_attn(fake, fake, fake, fake, fake, 5000, 1, 1, 1, 128, 128,
+    st = lib.velox_block_sparse_attn(fake, fake, fake, fake, fake, None, 5000, 1, 1, 1, 128, 128,
                                      ctypes.c_float(0.0), fake, None, fake, None)
     assert st == 2
-    # misaligned tensor -> invalid
-    st = lib.velox_block_sparse_attn(P(0x10002), fake, fake, None, None, 0, 1, 1, 1, 128, 128,
+    # a row order without a status word to report bad entries -> invalid
+    st = lib.velox_block_sparse_attn(fake, fake, fake, None, None, fake, 0, 1, 1, 1, 128, 128,
                                      ctypes.c_float(0.0), fake, None, None, None)
+    assert st == 1
+    lib.velox_route_schedule.restype = ctypes.c_int
+    assert lib.velox_route_schedule(None, 4, 10, fake, None) == 1
+    assert lib.velox_route_schedule(fake, 4, 5000, fake, None) == 2
+    # misaligned tensor -> invalid
+    st = lib.velox_block_sparse_attn(P(0x10002), fake, fake, None, None, None, 0, 1, 1, 1, 128,
+                                     128, ctypes.c_float(0.0), fake, None, None, None)
     assert st == 1
     # gilbert: W < H and W odd with H even are unsupported
     lib.velox_gilbert_order.restype = ctypes.c_int
