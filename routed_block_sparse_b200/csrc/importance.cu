@@ -5,14 +5,20 @@
 // the mean-query / mean-key inner product.
 //
 // Three launches:
-//   pool_kernel     streams Q and K once (the HBM-bound part: at the
-//                   chunk-48 shape K alone is 2.96 GB) and writes the fp32
-//                   block means qbar [H][N][d], kbar [H][M][d] to the
-//                   workspace.  One warp per 128 x 128 bf16 block, 16-byte
-//                   non-caching loads, 8 loads in flight per lane.
-//   logits_kernel   per (head, 64 history blocks): the N x 64 tile of
-//                   scale * qbar . kbar, written into p as raw logits.
-//   softmax_kernel  per (head, query block) row: max, sum of exp, normalise.
+//   pool_kernel          query blocks: fp32 means qbar [H][N][d] into the
+//                        workspace.  One warp per 128 x 128 bf16 block,
+//                        16-byte non-caching loads, 8 loads in flight per lane.
+//   pool_logits_kernel   streams K once (the HBM-bound part: 2.96 GB at the
+//                        chunk-48 shape).  A CTA takes a contiguous range of
+//                        one head's key blocks with that head's qbar in
+//                        shared memory; each warp pools one block and its two
+//                        half-warps dot the mean with half of the query rows
+//                        each; logits are staged in shared memory and written
+//                        into p row-contiguously.  No key means touch memory.
+//   softmax_kernel       per (head, query block) row: max, sum of exp,
+//                        normalise, in place.
+// When N > kFusedMaxN the key means go through the workspace instead
+// (pool_kernel on K, then logits_kernel).
 #include "common.cuh"
 
 namespace velox {
@@ -36,7 +42,7 @@ __device__ __forceinline__ void acc8(float (&a)[8], const uint4 &v) {
   a[6] += bf16_lo(v.w); a[7] += bf16_hi(v.w);
 }
 
-// Unit u < n_q: query block (h = u / N, i = u % N); else key block.
+// Unit u < n_q: block u of Q (means to qbar); else block u - n_q of K (to kbar).
 // Rows of a block are 256 bytes = 16 lanes x 16 bytes: lanes 0-15 take even
 // rows, lanes 16-31 odd rows; each lane sums 8 channels over 64 rows.
 __global__ void __launch_bounds__(256) pool_kernel(const uint16_t *__restrict__ Q,
@@ -134,6 +140,80 @@ __global__ void __launch_bounds__(256) logits_kernel(const float *__restrict__ q
   }
 }
 
+// Fused K pooling + logits.  Grid-stride over chunks of kFusedBlocks key
+// blocks of one head (chunk c: head c / cpr, blocks (c % cpr) * kFusedBlocks ..),
+// 256 threads, grid sized to the resident capacity.
+// Warp w of a CTA streams the 8 consecutive key blocks r0 + 8w .. r0 + 8w + 7
+// with no block-level barrier after the qbar load.  After the half-warp
+// exchange both halves hold the 8 channel sums of lane (l & 15); half-warp 0
+// computes the logits of query rows 0, 2, 4, ... and half-warp 1 of rows
+// 1, 3, 5, ..., each as 8 products plus a 16-lane shuffle reduction, staged
+// in the warp's own [N][8] shared-memory slice and written out row by row
+// (8 consecutive logits = 32 bytes per row) once the warp's blocks are done.
+constexpr int kFusedMaxN = 96;
+constexpr int kFusedWarps = 8;
+constexpr int kFusedPerWarp = 8;
+constexpr int kFusedBlocks = kFusedWarps * kFusedPerWarp;  // key blocks per CTA
+
+__global__ void __launch_bounds__(256) pool_logits_kernel(const uint16_t *__restrict__ K,
+                                                          const float *__restrict__ qbar, int H,
+                                                          int N, int M, float scale,
+                                                          float *__restrict__ p) {
+  extern __shared__ float4 fsm[];
+  float *qs = reinterpret_cast<float *>(fsm);  // [N][D] means of the chunk's head
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float *lg = qs + N * D + warp * N * kFusedPerWarp;  // this warp's [N][8] logits
+  const int col = (lane & 15) * 8;
+  const int row0 = lane >> 4;
+  const float cs = scale * (1.0f / BT);  // logit = scale * qbar . (sum / b)
+  const int cpr = (M + kFusedBlocks - 1) / kFusedBlocks;
+  for (int c = blockIdx.x; c < H * cpr; c += gridDim.x) {
+  const int h = c / cpr;
+  __syncthreads();  // every warp is done with the previous chunk's qbar
+  for (int e = threadIdx.x; e < N * D / 4; e += blockDim.x)
+    fsm[e] = reinterpret_cast<const float4 *>(qbar + (size_t)h * N * D)[e];
+  __syncthreads();
+  const int rw = (c - h * cpr) * kFusedBlocks + warp * kFusedPerWarp;  // first block of the warp
+  for (int k = 0; k < kFusedPerWarp; ++k) {
+    const int rb = rw + k;
+    if (rb >= M) break;  // uniform across the warp
+    float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const uint16_t *src = K + ((size_t)h * M + rb) * BT * D + row0 * D + col;
+#pragma unroll 1
+    for (int r = 0; r < BT / 2; r += 16) {
+      uint4 v[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) v[q] = ld_stream(src + (size_t)(r + q) * 2 * D);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) acc8(a, v[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) a[q] += __shfl_xor_sync(0xffffffffu, a[q], 16);
+    // same trip count in both half-warps (the shuffles span the whole warp)
+    for (int ii = 0; ii < (N + 1) / 2; ++ii) {
+      const int i = 2 * ii + row0;
+      const int iq = i < N ? i : N - 1;  // odd N: half-warp 1 repeats a row, unused
+      const float4 q0 = *reinterpret_cast<const float4 *>(qs + iq * D + col);
+      const float4 q1 = *reinterpret_cast<const float4 *>(qs + iq * D + col + 4);
+      float d = q0.x * a[0];
+      d = fmaf(q0.y, a[1], d); d = fmaf(q0.z, a[2], d); d = fmaf(q0.w, a[3], d);
+      d = fmaf(q1.x, a[4], d); d = fmaf(q1.y, a[5], d); d = fmaf(q1.z, a[6], d);
+      d = fmaf(q1.w, a[7], d);
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+      if ((lane & 15) == 0 && i < N) lg[i * kFusedPerWarp + k] = d * cs;
+    }
+  }
+  __syncwarp();
+  const int nb = min(kFusedPerWarp, M - rw);
+  for (int e = lane; e < N * kFusedPerWarp; e += 32) {
+    const int i = e / kFusedPerWarp, k = e - i * kFusedPerWarp;
+    if (k < nb) p[((size_t)h * N + i) * M + rw + k] = lg[e];
+  }
+  __syncwarp();
+  }
+}
+
 __device__ __forceinline__ void merge_ms(float &m, float &s, float m2, float s2) {
   float mm = fmaxf(m, m2);
   if (mm == -INFINITY) return;
@@ -190,15 +270,30 @@ cudaError_t launch_importance(const uint16_t *Q, const uint16_t *K, int H, int N
                               float scale, float *p, void *ws, cudaStream_t stream) {
   float *qbar = static_cast<float *>(ws);
   float *kbar = qbar + (size_t)H * N * D;
+  const bool fused = N <= kFusedMaxN;
   const int n_q = H * N;
-  const int n_units = H * (N + M);
+  const int n_units = fused ? n_q : H * (N + M);
   int grid = (n_units + 7) / 8;
   if (grid > 148 * 8 * 4) grid = 148 * 8 * 4;
   pool_kernel<<<grid, 256, 0, stream>>>(Q, K, n_q, n_units, qbar, kbar);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dim3 lg((M + LG_R - 1) / LG_R, H);
-  logits_kernel<<<lg, 256, 0, stream>>>(qbar, kbar, N, M, scale, p);
+  if (fused) {
+    const size_t smem = (size_t)N * (D + kFusedWarps * kFusedPerWarp) * sizeof(float);
+    if (smem > 48 * 1024) {
+      e = cudaFuncSetAttribute(pool_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    const int chunks = H * ((M + kFusedBlocks - 1) / kFusedBlocks);
+    int per_sm = (int)((220 * 1024) / (smem + 1024));
+    per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
+    const int grid_f = chunks < 148 * per_sm ? chunks : 148 * per_sm;
+    pool_logits_kernel<<<grid_f, 256, smem, stream>>>(K, qbar, H, N, M, scale, p);
+  } else {
+    dim3 lg((M + LG_R - 1) / LG_R, H);
+    logits_kernel<<<lg, 256, 0, stream>>>(qbar, kbar, N, M, scale, p);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   softmax_kernel<<<H * N, 256, 0, stream>>>(p, M);
