@@ -55,3 +55,35 @@ def dense_attention_block(q, Kh, Vh, b: int, scale: float = 0.0):
     """Dense attention of one query block over all M history blocks."""
     M = Kh.shape[0] // b
     return routed_attention_block(q, Kh, Vh, range(M), b, scale)
+
+
+def two_phase_attention_block(q: np.ndarray, Kh: np.ndarray, Vh: np.ndarray,
+                              tiles: Iterable[int], Kc: np.ndarray, Vc: np.ndarray, b: int,
+                              scale: float = 0.0) -> Tuple[np.ndarray, np.ndarray]:
+    """Routed history tiles plus the current chunk's own keys, one softmax.
+
+    The pages' kernel runs a "two-phase tile loop" (digest of arXiv
+    2610.22311, "Reproducibility"): the routed history tiles of the KV cache
+    and the tiles of the chunk being generated.  Reading: a query token
+    attends to every token of its routed history tiles and to every token of
+    the current chunk (Kc, Vc: [N_cur*b][d] of the same head), with one
+    normaliser over both.  Returns (O [b][d], lse [b]) in fp64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    d = q.shape[1]
+    if scale <= 0.0:
+        scale = 1.0 / math.sqrt(d)
+    tiles = sorted(set(int(t) for t in tiles))
+    parts_k = [np.asarray(Kh[t * b:(t + 1) * b], dtype=np.float64) for t in tiles]
+    parts_v = [np.asarray(Vh[t * b:(t + 1) * b], dtype=np.float64) for t in tiles]
+    parts_k.append(np.asarray(Kc, dtype=np.float64))
+    parts_v.append(np.asarray(Vc, dtype=np.float64))
+    k = np.concatenate(parts_k)
+    v = np.concatenate(parts_v)
+    if k.shape[0] == 0:
+        return np.zeros_like(q), np.full(q.shape[0], -np.inf)
+    x = (q @ k.T) * scale
+    m = x.max(axis=1, keepdims=True)
+    e = np.exp(x - m)
+    l = e.sum(axis=1, keepdims=True)
+    return (e @ v) / l, m[:, 0] + np.log(l[:, 0])

@@ -80,3 +80,37 @@ def test_empty_route():
     q, K, V = _data(4, 3)
     O, lse = at.routed_attention_block(q, K, V, [], B)
     assert np.all(O == 0) and np.all(np.isneginf(lse))
+
+
+def test_two_phase_equals_library_attention_over_concatenated_keys():
+    q, K, V = _data(5, 6)
+    r = np.random.default_rng(5)
+    Kc = r.standard_normal((3 * B, D))
+    Vc = r.standard_normal((3 * B, D))
+    tiles = [4, 1]
+    O, lse = at.two_phase_attention_block(q, K, V, tiles, Kc, Vc, B)
+    idx = np.concatenate([np.arange(t * B, (t + 1) * B) for t in sorted(tiles)])
+    kk = np.concatenate([K[idx], Kc])
+    vv = np.concatenate([V[idx], Vc])
+    assert np.allclose(O, _sdpa(q, kk, vv), rtol=0, atol=1e-12)
+    x = torch.from_numpy(q @ kk.T / math.sqrt(D))
+    assert np.allclose(lse, torch.logsumexp(x, dim=1).numpy(), rtol=0, atol=1e-12)
+
+
+def test_two_phase_is_the_merge_of_its_two_phases():
+    # softmax over a union of disjoint key sets = the two partial results
+    # merged with weights exp(lse_part - lse_all)
+    q, K, V = _data(6, 7)
+    r = np.random.default_rng(6)
+    Kc = r.standard_normal((2 * B, D))
+    Vc = r.standard_normal((2 * B, D))
+    tiles = [0, 3, 6]
+    Oh, lh = at.routed_attention_block(q, K, V, tiles, B)
+    Oc, lc = at.routed_attention_block(q, Kc, Vc, [0, 1], B)
+    O, lse = at.two_phase_attention_block(q, K, V, tiles, Kc, Vc, B)
+    assert np.allclose(lse, np.logaddexp(lh, lc), rtol=0, atol=1e-12)
+    want = np.exp(lh - lse)[:, None] * Oh + np.exp(lc - lse)[:, None] * Oc
+    assert np.allclose(O, want, rtol=0, atol=1e-12)
+    # no history tiles: plain attention over the current chunk
+    O0, _ = at.two_phase_attention_block(q, K, V, [], Kc, Vc, B)
+    assert np.allclose(O0, Oc, rtol=0, atol=1e-12)
