@@ -26,11 +26,16 @@ Modules and the passages they follow:
                  Eq. 12-14; onedev.kr summary, "How it differs").
 - ``attention``  attention over exactly the tokens of the routed 128-token KV
                  tiles (digest, "Core method", Eq. 15; project page, "Why the
-                 route is a block, not a token").
+                 route is a block, not a token"), and its two-phase form with
+                 the current chunk's own keys (digest, "Reproducibility").
+- ``geometry``   frustum-slab overlap g_{i,r} and coverage rho_i, the inputs
+                 of the route build (project page, "02 · Method", steps 01-02;
+                 digest, "Method steps", Eq. 7-8; onedev.kr summary, "How it
+                 differs").
 
 Every function here is pinned by the ``-m "not gpu"`` tests in
 ``tests/test_oracle_*.py`` against invariants, closed forms, textbook routines
 and brute force, not against itself.
 """
 
-from . import gilbert, importance, route, attention  # noqa: F401
+from . import gilbert, importance, route, attention, geometry  # noqa: F401
