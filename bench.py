@@ -396,6 +396,83 @@ def _e2e(args, wl, inp, layer, dev, stream, flops_step, world):
             "d2h_bytes_per_step": d2h}
 
 
+def run_sweep(args):
+    """History-length sweep (chunk-48 per-chunk shape, M cache blocks): the
+    routed path and the library's own dense kernel over the same cache, one
+    JSON line per M.  Not the bench line; for the scaling table."""
+    from routed_block_sparse_b200.pipeline import layer_for
+    from synth import make_inputs, sweep_workload
+    from synth.configs import SWEEP_M
+
+    for M in SWEEP_M:
+        wl = sweep_workload(M)
+        inp = make_inputs(wl, "cuda")
+        layer = layer_for(wl)
+        layer.forward(inp.Q, inp.K, inp.V, inp.g, inp.covered)
+        torch.cuda.synchronize()
+        tiles = float(layer.route_len.sum().item())
+        out = {"sweep_M": M, "mean_route_len": tiles / (wl.heads * wl.n_q_blocks)}
+        for mode in ("routed", "dense"):
+            n_t = tiles if mode == "routed" else float(wl.heads * wl.n_q_blocks * M)
+            for _ in range(3):
+                layer.attend(inp.Q, inp.K, inp.V, dense=(mode == "dense"))
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            reps = 20
+            a.record()
+            for _ in range(reps):
+                layer.attend(inp.Q, inp.K, inp.V, dense=(mode == "dense"))
+            b.record()
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / reps
+            out[f"{mode}_us"] = ms * 1e3
+            out[f"{mode}_tflops"] = 4.0 * 128 ** 3 * n_t / (ms * 1e-3) / 1e12
+        out["speedup_routed_vs_dense"] = out["dense_us"] / out["routed_us"]
+        print(json.dumps(out), flush=True)
+        del inp, layer
+        torch.cuda.empty_cache()
+
+
+def run_layers(args):
+    """Full denoising step at chunk 48: `args.layers` layers with independent
+    per-layer inputs (seeded per layer), regenerated into reused buffers
+    between layers outside the timed spans (40 layers of K+V would be 236 GB).
+    Per layer the importance, route build + schedule and attention run back to
+    back on one stream; the summed times are reported."""
+    from routed_block_sparse_b200.pipeline import layer_for
+    from synth import config, make_inputs
+
+    wl0 = config(5, 0)
+    layer = layer_for(wl0)
+    inp = make_inputs(wl0, "cuda")
+    stream = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    t_route = t_attn = 0.0
+    tiles = 0.0
+    status = 0
+    for li in range(args.layers):
+        inp = make_inputs(config(5, li), "cuda", out=inp)
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        layer.importance(inp.Q, inp.K, stream)
+        layer.route(inp.g, inp.covered, stream=stream)
+        ev[1].record(stream)
+        layer.attend(inp.Q, inp.K, inp.V, stream=stream)
+        ev[2].record(stream)
+        torch.cuda.synchronize()
+        t_route += ev[0].elapsed_time(ev[1])
+        t_attn += ev[1].elapsed_time(ev[2])
+        tiles += float(layer.route_len.sum().item())
+        status |= layer.status()
+    flops = 4.0 * 128 ** 3 * tiles
+    print(json.dumps({"mode": "layers", "layers": args.layers,
+                      "route_build_ms_total": t_route, "attention_ms_total": t_attn,
+                      "attention_tflops": flops / (t_attn * 1e-3) / 1e12,
+                      "route_share": t_route / (t_route + t_attn), "dev_status": status,
+                      "note": "importance + route build + schedule per layer counted as route build"}),
+          flush=True)
+
+
 def _attn_source_hash() -> str:
     import hashlib
     p = os.path.join(ROOT, "routed_block_sparse_b200", "csrc", "attn.cu")
@@ -411,6 +488,11 @@ def main():
     ap.add_argument("--impl", default="velox", choices=["velox", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="history-length sweep: routed vs dense attention per M (extra lines)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="full-step mode: this many chunk-48 layers with per-layer inputs "
+                         "(extra line with the summed route-build and attention times)")
     ap.add_argument("--heads", type=int, default=0,
                     help="run a reduced head count (profiler captures only)")
     args = ap.parse_args()
@@ -423,6 +505,12 @@ def main():
         return
     world, rank, local = _dist_setup()
     try:
+        if args.sweep:
+            run_sweep(args)
+            return
+        if args.layers:
+            run_layers(args)
+            return
         run_velox(args, world, rank, local)
     finally:
         if world > 1:

@@ -165,10 +165,17 @@ __global__ void __launch_bounds__(kThreads) route_kernel(RouteArgs a) {
     for (int shift = 56; shift >= 0; shift -= 8) {
       for (int k = tid; k < 256; k += kThreads) s_hist[k] = 0;
       __syncthreads();
-      for (int r = tid; r < M; r += kThreads) {
-        if (r >= pb && r < pe) continue;
-        const uint64_t u = order_key(keys[r]);
-        if ((u & mask) == prefix) atomicAdd(&s_hist[(u >> shift) & 255u], 1);
+      // warp-aggregated: keys mostly share their leading digits, so one
+      // atomic per distinct digit per warp instead of one per key
+      for (int base = 0; base < M; base += kThreads) {
+        const int r = base + tid;
+        int digit = -1;
+        if (r < M && !(r >= pb && r < pe)) {
+          const uint64_t u = order_key(keys[r]);
+          if ((u & mask) == prefix) digit = static_cast<int>((u >> shift) & 255u);
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, digit);
+        if (digit >= 0 && (tid & 31) == __ffs(peers) - 1) atomicAdd(&s_hist[digit], __popc(peers));
       }
       __syncthreads();
       if (tid < 32) {
