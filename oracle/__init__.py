@@ -33,9 +33,14 @@ Modules and the passages they follow:
                  digest, "Method steps", Eq. 7-8; onedev.kr summary, "How it
                  differs").
 
+- ``audit``      the geometry-model consistency audit: R_geo, R_50, top-80
+                 recall with and without fusion, changed blocks (project
+                 page, "03 · Results"; digest, results table; onedev.kr
+                 summary, "Results").
+
 Every function here is pinned by the ``-m "not gpu"`` tests in
 ``tests/test_oracle_*.py`` against invariants, closed forms, textbook routines
 and brute force, not against itself.
 """
 
-from . import gilbert, importance, route, attention, geometry  # noqa: F401
+from . import gilbert, importance, route, attention, geometry, audit  # noqa: F401
