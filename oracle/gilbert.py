@@ -126,8 +126,30 @@ def global_order(T: int, H: int, W: int, n_chunks: int, b: int):
     return rank_of_cell, cell_of_rank, rank_of_cell // b
 
 
+def thw_linear_order(T: int, H: int, W: int, n_chunks: int, b: int):
+    """The THW-linear order the pages compare against (project page, figure
+    "THW-linear against global Gilbert order"): tokens flattened frame by
+    frame, each frame row by row, rank(f, y, x) = (f * H + y) * W + x.
+    Same return convention as global_order."""
+    if min(T, H, W, b) < 1:
+        raise ValueError("non-positive lattice size")
+    if (T * H * W) % b != 0:
+        raise ValueError("T*H*W must be a multiple of the block size")
+    F = n_chunks * T
+    rank = np.empty((F, H, W), dtype=np.int64)
+    for f in range(F):
+        for y in range(H):
+            for x in range(W):
+                rank[f, y, x] = (f * H + y) * W + x
+    rank_of_cell = rank.reshape(-1)
+    cell_of_rank = np.empty_like(rank_of_cell)
+    cell_of_rank[rank_of_cell] = np.arange(rank_of_cell.size)
+    return rank_of_cell, cell_of_rank, rank_of_cell // b
+
+
 def neighbour_blocks(T: int, H: int, W: int, n_chunks: int, b: int,
-                     q_chunk: int, cache_first_block: int, n_cache_blocks: int):
+                     q_chunk: int, cache_first_block: int, n_cache_blocks: int,
+                     layout: str = "gilbert"):
     """26-neighbour safeguard blocks of every query block of chunk q_chunk.
 
     Reading of "Gilbert 26-neighbour blocks" (digest, "Method steps", Eq. 14;
@@ -137,9 +159,11 @@ def neighbour_blocks(T: int, H: int, W: int, n_chunks: int, b: int,
     blocks inside the cache range are kept, as cache ids
     (global block id - cache_first_block), ascending.
 
+    layout "gilbert" (the global Gilbert order) or "thw" (THW-linear).
     Returns a list (one entry per query block of the chunk) of int lists.
     """
-    _, _, block_of_cell = global_order(T, H, W, n_chunks, b)
+    order = {"gilbert": global_order, "thw": thw_linear_order}[layout]
+    _, _, block_of_cell = order(T, H, W, n_chunks, b)
     F = n_chunks * T
     blk = block_of_cell.reshape(F, H, W)
     per_chunk = T * H * W // b
