@@ -16,6 +16,13 @@
  *   4. velox_block_sparse_attn  online-softmax attention over only the routed
  *                               128-token KV tiles (tcgen05 / TMEM / TMA).
  *
+ * Around it: velox_two_phase_attn (routed history plus the current chunk's
+ * own tiles under one softmax), velox_slab_overlap and velox_coverage (the
+ * geometric inputs g and the coverage flags), velox_route_audit (the
+ * geometry-model consistency counts), velox_thw_linear_order (the raster
+ * order the pages compare the Gilbert order with), velox_route_schedule
+ * (longest-route-first row order) and velox_block_importance_noalloc.
+ *
  * Conventions shared by every call
  * --------------------------------
  * - Every pointer argument is a DEVICE pointer, owned by the caller, unless
@@ -75,6 +82,7 @@ typedef enum {
 #define VELOX_DEV_WAIT_TIMEOUT   0x20  /* bounded mbarrier wait gave up        */
 #define VELOX_DEV_ROUTE_CAPACITY 0x40  /* route row longer than R_max: cut     */
 #define VELOX_DEV_BAD_ROW_ORDER  0x80  /* row_order entry outside [0, H*N)      */
+#define VELOX_DEV_BAD_CAMERA     0x100 /* slab camera index outside [0, n_cams)  */
 
 /* Supported sizes of the importance and attention calls. */
 #define VELOX_HEAD_DIM   128
@@ -135,6 +143,26 @@ VELOX_API velox_status velox_gilbert_order(int T, int H, int W, int n_chunks, in
                                  int32_t *cell_of_rank, int32_t *block_of_cell,
                                  int32_t *nbr_ids, int32_t *nbr_cnt, int S_max,
                                  int32_t *dev_status, velox_stream_t stream);
+
+/*
+ * velox_thw_linear_order -- the THW-linear (raster) order that the pages set
+ * against the global Gilbert order, with the same outputs.
+ *
+ * Defined by: project page, figure "THW-linear against global Gilbert order"
+ * (toy latent H = 3, W = 4, block size 2) and "Keeping neighbours adjacent
+ * in the block order".
+ *
+ * rank(f, y, x) = (f * H + y) * W + x: the rank of a cell is its cell index,
+ * a block is b_tok consecutive raster cells.  Arguments, layouts, the
+ * safeguard definition and errors are those of velox_gilbert_order, except
+ * that any H and W are accepted (T*H*W % b_tok == 0 still required).
+ */
+VELOX_API velox_status velox_thw_linear_order(int T, int H, int W, int n_chunks, int b_tok,
+                                              int q_chunk, int cache_first_block,
+                                              int n_cache_blocks, int32_t *rank_of_cell,
+                                              int32_t *cell_of_rank, int32_t *block_of_cell,
+                                              int32_t *nbr_ids, int32_t *nbr_cnt, int S_max,
+                                              int32_t *dev_status, velox_stream_t stream);
 
 /*
  * velox_workspace_size -- bytes of device workspace that
@@ -285,6 +313,124 @@ VELOX_API velox_status velox_block_sparse_attn(const velox_bf16 *Q, const velox_
                                                float softmax_scale, velox_bf16 *O,
                                                float *lse, int32_t *dev_status,
                                                velox_stream_t stream);
+
+/*
+ * velox_two_phase_attn -- routed history attention and the current chunk's
+ * own keys in one softmax.
+ *
+ * Defined by: digest, "Reproducibility" (the two-phase tile loop) and
+ * "Core method" (Eq. 15); project page, "02 · Method", step 04.  Reading:
+ * every query token of block i attends to the tokens of its routed history
+ * tiles (as velox_block_sparse_attn) and to all N_cur*b_tok tokens of the
+ * current chunk, with one normaliser over both phases:
+ *   O = sum over u in (routed history tokens) U (current tokens) of
+ *       softmax_u(softmax_scale * q . k_u) v_u,   lse = log sum exp(...).
+ *
+ * K_cur, V_cur [H][N_cur*b][d] bf16 (16-byte aligned), N_cur > 0; all other
+ * arguments, layouts, limits and device errors as velox_block_sparse_attn
+ * (route_ids == NULL: all M history tiles).
+ */
+VELOX_API velox_status velox_two_phase_attn(const velox_bf16 *Q, const velox_bf16 *K,
+                                            const velox_bf16 *V, const int32_t *route_ids,
+                                            const int32_t *route_len,
+                                            const int32_t *row_order, int R_max,
+                                            const velox_bf16 *K_cur, const velox_bf16 *V_cur,
+                                            int N_cur, int H, int N, int M, int d, int b_tok,
+                                            float softmax_scale, velox_bf16 *O, float *lse,
+                                            int32_t *dev_status, velox_stream_t stream);
+
+/* A pinhole camera in latent-token units: pixel (u, v) at depth z is the
+ * camera-frame point ((u - cx) / fx * z, (v - cy) / fy * z, z); the world
+ * point is C + R x (R: world-from-camera rotation, row-major). */
+typedef struct {
+  float fx, fy, cx, cy;
+  float R[9];
+  float C[3];
+} velox_camera;
+
+/* A frustum slab: token rectangle [u0, u1) x [v0, v1) of camera `cam` and
+ * the depth interval [zlo, zhi]; `valid` = 0 marks a block without reliable
+ * geometry. */
+typedef struct {
+  float u0, u1, v0, v1, zlo, zhi;
+  int32_t cam;
+  int32_t valid;
+} velox_slab;
+
+/*
+ * velox_slab_overlap -- g[i][r], the world-space overlap of query slab i and
+ * history slab r.
+ *
+ * Defined by: project page, "02 · Method", glossary entry for g (overlap, IoU,
+ * of the slabs in world space); digest, "Prerequisites" (frustum slab, OBB
+ * overlap) and "Method steps", step three (Eq. 7).  Each slab is the
+ * camera-facing oriented box with the camera's axes, centred on the ray
+ * through the rectangle centre at the mid depth zm, half extents
+ * (u1-u0)/(2 fx) zm, (v1-v0)/(2 fy) zm, (zhi-zlo)/2.  The intersection is
+ * counted on the grid^3 cell centres of the query box:
+ *   g = inter / (vol_i + vol_r - inter),  inter = vol_i * inside / grid^3;
+ * an invalid history slab gives 0.
+ *
+ * cams [n_cams], q_slabs [N], h_slabs [M] (device), g [N][M] fp32 out.
+ * 1 <= grid <= 32, N <= 65535 (VELOX_ERR_UNSUPPORTED otherwise).  A slab whose camera index is out of range gives 0 and
+ * flags VELOX_DEV_BAD_CAMERA.
+ */
+VELOX_API velox_status velox_slab_overlap(const velox_camera *cams, int n_cams,
+                                          const velox_slab *q_slabs, int N,
+                                          const velox_slab *h_slabs, int M, int grid,
+                                          float *g, int32_t *dev_status,
+                                          velox_stream_t stream);
+
+/*
+ * velox_coverage -- rho[i], the fraction of query block i's tokens whose
+ * warped depth falls inside a valid past slab, and covered[i] = rho >= eta.
+ *
+ * Defined by: digest, "Method steps", step three (Eq. 8: coverage and the
+ * eta_cov = 0.9 threshold); onedev.kr summary, "How it differs" (a token is
+ * covered when its multiwarp depth falls inside a valid past slab).
+ * A token (u, v, z) of query block i (camera q_slabs[i].cam) is back-projected
+ * and projected into each valid history slab's camera; it is covered when it
+ * lands in the slab's rectangle at a depth in [zlo, zhi].  z <= 0 (a hole) is
+ * never covered.
+ *
+ * q_uvz [N][b][3] fp32 (u, v, z per token), 1 <= b <= 128; rho [N] fp32,
+ * covered [N] uint8 out.
+ */
+VELOX_API velox_status velox_coverage(const velox_camera *cams, int n_cams,
+                                      const velox_slab *q_slabs, const float *q_uvz, int N,
+                                      int b, const velox_slab *h_slabs, int M, float eta,
+                                      float *rho, uint8_t *covered, int32_t *dev_status,
+                                      velox_stream_t stream);
+
+/*
+ * velox_route_audit -- the geometry-model consistency audit, as six integer
+ * counts per (head, query block) row.
+ *
+ * Defined by: project page, "03 · Results", "Geometry and the model agree"
+ * (R_geo: positive-overlap blocks in the model's own top-50; fusion at
+ * lambda = 2 raising the top-80 recall of positive-overlap blocks while
+ * changing few selected blocks); digest, results table, row
+ * "geometry-model importance consistency audit" (R_geo and the top-50
+ * agreement R_50 against the random expectation 50/143); onedev.kr summary,
+ * "Results".
+ *
+ * pos = {r : g[i][r] > tau}; top_K(x) = the K largest x_r, ties to the lower
+ * id (all M when K >= M); fused = p (1 + lambda min(g / g_ref, 1) [g > tau])
+ * in fp64 on every row.  counts[row][0..5] =
+ *   |pos|, |pos & top_kgeo(p)|, |top_kgeo(g) & top_kgeo(p)|,
+ *   |pos & top_kfuse(p)|, |pos & top_kfuse(fused)|,
+ *   |top_kfuse(fused) - top_kfuse(p)|.
+ * Pooled over rows: R_geo = sum c1 / sum c0, R_50 = sum c2 / (rows min(kgeo, M)),
+ * top-kfuse recall = sum c3 (model) or sum c4 (fused) over sum c0,
+ * changed = sum c5 / (rows min(kfuse, M)).
+ *
+ * p [H][N][M] fp32, g [N][M] fp32 (device), prm: host pointer (lambda, tau,
+ * g_ref used), counts [H][N][6] int32 out.  M <= 4096 (VELOX_ERR_UNSUPPORTED
+ * otherwise); k_geo, k_fuse >= 1.
+ */
+VELOX_API velox_status velox_route_audit(const float *p, const float *g, int H, int N, int M,
+                                         const velox_route_params *prm, int k_geo, int k_fuse,
+                                         int32_t *counts, velox_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -30,6 +30,7 @@ DEV_BAD_SAFEGUARD = 0x10
 DEV_WAIT_TIMEOUT = 0x20
 DEV_ROUTE_CAPACITY = 0x40
 DEV_BAD_ROW_ORDER = 0x80
+DEV_BAD_CAMERA = 0x100
 HEAD_DIM = 128
 BLOCK_TOK = 128
 MAX_BLOCKS = 65536
@@ -39,7 +40,8 @@ NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 EXPORTS = ("velox_status_string", "velox_abi_version", "velox_gilbert_order",
            "velox_workspace_size", "velox_block_importance", "velox_route_build",
            "velox_block_sparse_attn", "velox_block_importance_noalloc",
-           "velox_route_schedule")
+           "velox_route_schedule", "velox_two_phase_attn", "velox_slab_overlap",
+           "velox_coverage", "velox_route_audit", "velox_thw_linear_order")
 
 
 class VeloxError(RuntimeError):
@@ -67,6 +69,8 @@ def _load() -> ctypes.CDLL:
     lib.velox_abi_version.argtypes = []
     lib.velox_gilbert_order.restype = I
     lib.velox_gilbert_order.argtypes = [I, I, I, I, I, I, I, I, P, P, P, P, P, I, P, P]
+    lib.velox_thw_linear_order.restype = I
+    lib.velox_thw_linear_order.argtypes = [I, I, I, I, I, I, I, I, P, P, P, P, P, I, P, P]
     lib.velox_workspace_size.restype = I
     lib.velox_workspace_size.argtypes = [I, I, I, I, ctypes.POINTER(ctypes.c_size_t)]
     lib.velox_block_importance.restype = I
@@ -80,6 +84,15 @@ def _load() -> ctypes.CDLL:
     lib.velox_route_schedule.argtypes = [P, I, I, P, P]
     lib.velox_block_sparse_attn.restype = I
     lib.velox_block_sparse_attn.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, P]
+    lib.velox_slab_overlap.restype = I
+    lib.velox_slab_overlap.argtypes = [P, I, P, I, P, I, I, P, P, P]
+    lib.velox_coverage.restype = I
+    lib.velox_coverage.argtypes = [P, I, P, P, I, I, P, I, F, P, P, P, P]
+    lib.velox_route_audit.restype = I
+    lib.velox_route_audit.argtypes = [P, P, I, I, I, ctypes.POINTER(RouteParams), I, I, P, P]
+    lib.velox_two_phase_attn.restype = I
+    lib.velox_two_phase_attn.argtypes = [P, P, P, P, P, P, I, P, P, I, I, I, I, I, I, F, P, P, P,
+                                         P]
     return lib
 
 
@@ -122,6 +135,17 @@ def velox_gilbert_order(T, H, W, n_chunks, b_tok, q_chunk=0, cache_first_block=0
                                   _ptr(block_of_cell), _ptr(nbr_ids), _ptr(nbr_cnt), S_max,
                                   _ptr(dev_status), _stream(stream))
     _check("velox_gilbert_order", st)
+
+
+def velox_thw_linear_order(T, H, W, n_chunks, b_tok, q_chunk=0, cache_first_block=0,
+                           n_cache_blocks=0, rank_of_cell=None, cell_of_rank=None,
+                           block_of_cell=None, nbr_ids=None, nbr_cnt=None, S_max=0,
+                           dev_status=None, stream=None):
+    st = _lib.velox_thw_linear_order(T, H, W, n_chunks, b_tok, q_chunk, cache_first_block,
+                                     n_cache_blocks, _ptr(rank_of_cell), _ptr(cell_of_rank),
+                                     _ptr(block_of_cell), _ptr(nbr_ids), _ptr(nbr_cnt), S_max,
+                                     _ptr(dev_status), _stream(stream))
+    _check("velox_thw_linear_order", st)
 
 
 def velox_workspace_size(H, N, M, d=HEAD_DIM) -> int:
@@ -174,3 +198,36 @@ def velox_block_sparse_attn(Q, K, V, route_ids, route_len, R_max, H, N, M, d, b_
 def route_params(lam=2.0, tau=0.1, g_ref=0.2, theta_cov=0.9, theta_unc=0.9, k_cov=80,
                  k_unc=150) -> RouteParams:
     return RouteParams(lam, tau, g_ref, theta_cov, theta_unc, k_cov, k_unc)
+
+
+def velox_two_phase_attn(Q, K, V, route_ids, route_len, R_max, K_cur, V_cur, N_cur, H, N, M, d,
+                         b_tok, softmax_scale, O, lse=None, dev_status=None, stream=None,
+                         row_order=None):
+    st = _lib.velox_two_phase_attn(_ptr(Q), _ptr(K), _ptr(V), _ptr(route_ids), _ptr(route_len),
+                                   _ptr(row_order), R_max, _ptr(K_cur), _ptr(V_cur), N_cur, H, N,
+                                   M, d, b_tok, float(softmax_scale), _ptr(O), _ptr(lse),
+                                   _ptr(dev_status), _stream(stream))
+    _check("velox_two_phase_attn", st)
+
+
+# velox_camera: 16 fp32 (fx, fy, cx, cy, R row-major, C); velox_slab: 6 fp32
+# (u0, u1, v0, v1, zlo, zhi) then int32 cam, int32 valid.  Tensors of those
+# layouts (camera [n][16] float32, slab [n][8] int32 view) are passed as is.
+def velox_slab_overlap(cams, n_cams, q_slabs, N, h_slabs, M, grid, g, dev_status, stream=None):
+    st = _lib.velox_slab_overlap(_ptr(cams), n_cams, _ptr(q_slabs), N, _ptr(h_slabs), M, grid,
+                                 _ptr(g), _ptr(dev_status), _stream(stream))
+    _check("velox_slab_overlap", st)
+
+
+def velox_coverage(cams, n_cams, q_slabs, q_uvz, N, b, h_slabs, M, eta, rho, covered, dev_status,
+                   stream=None):
+    st = _lib.velox_coverage(_ptr(cams), n_cams, _ptr(q_slabs), _ptr(q_uvz), N, b, _ptr(h_slabs),
+                             M, float(eta), _ptr(rho), _ptr(covered), _ptr(dev_status),
+                             _stream(stream))
+    _check("velox_coverage", st)
+
+
+def velox_route_audit(p, g, H, N, M, prm, k_geo, k_fuse, counts, stream=None):
+    st = _lib.velox_route_audit(_ptr(p), _ptr(g), H, N, M, ctypes.byref(prm), k_geo, k_fuse,
+                                _ptr(counts), _stream(stream))
+    _check("velox_route_audit", st)

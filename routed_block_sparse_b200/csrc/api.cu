@@ -12,7 +12,8 @@ namespace velox {
 cudaError_t launch_gilbert(int T, int H, int W, int n_chunks, int b, int q_chunk,
                            int cache_first, int n_cache, int32_t *rank_of_cell,
                            int32_t *cell_of_rank, int32_t *block_of_cell, int32_t *nbr_ids,
-                           int32_t *nbr_cnt, int S_max, int32_t *dev_status, cudaStream_t stream);
+                           int32_t *nbr_cnt, int S_max, int thw, int32_t *dev_status,
+                           cudaStream_t stream);
 size_t importance_workspace_bytes(int H, int N, int M);
 cudaError_t launch_importance(const uint16_t *Q, const uint16_t *K, int H, int N, int M,
                               float scale, float *p, void *ws, cudaStream_t stream);
@@ -27,9 +28,21 @@ cudaError_t launch_schedule(const int32_t *route_len, int rows, int R_max, int32
                             cudaStream_t stream);
 cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                         const int32_t *route_ids, const int32_t *route_len,
-                        const int32_t *row_order, int R_max, int H,
-                        int N, int M, float softmax_scale, uint16_t *O, float *lse,
-                        int32_t *dev_status, cudaStream_t stream, bool *map_failed);
+                        const int32_t *row_order, int R_max, const uint16_t *K_cur,
+                        const uint16_t *V_cur, int N_cur, int H, int N, int M,
+                        float softmax_scale, uint16_t *O, float *lse, int32_t *dev_status,
+                        cudaStream_t stream, bool *map_failed);
+cudaError_t launch_slab_overlap(const velox_camera *cams, int n_cams, const velox_slab *qs, int N,
+                                const velox_slab *hs, int M, int G, float *g,
+                                int32_t *dev_status, cudaStream_t stream);
+cudaError_t launch_coverage(const velox_camera *cams, int n_cams, const velox_slab *qs,
+                            const float *q_uvz, int N, int b, const velox_slab *hs, int M,
+                            float eta, float *rho, uint8_t *covered, int32_t *dev_status,
+                            cudaStream_t stream);
+int audit_max_blocks();
+cudaError_t launch_audit(const float *p, const float *g, int H, int N, int M, double lam,
+                         double tau, double g_ref, int k_geo, int k_fuse, int32_t *counts,
+                         cudaStream_t stream);
 }  // namespace velox
 
 namespace {
@@ -90,14 +103,18 @@ const char *velox_status_string(velox_status s) {
 
 int velox_abi_version(void) { return 101; }
 
-velox_status velox_gilbert_order(int T, int H, int W, int n_chunks, int b_tok, int q_chunk,
-                                 int cache_first_block, int n_cache_blocks,
-                                 int32_t *rank_of_cell, int32_t *cell_of_rank,
-                                 int32_t *block_of_cell, int32_t *nbr_ids, int32_t *nbr_cnt,
-                                 int S_max, int32_t *dev_status, velox_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+velox_status order_common(int T, int H, int W, int n_chunks, int b_tok, int q_chunk,
+                          int cache_first_block, int n_cache_blocks, int32_t *rank_of_cell,
+                          int32_t *cell_of_rank, int32_t *block_of_cell, int32_t *nbr_ids,
+                          int32_t *nbr_cnt, int S_max, int thw, int32_t *dev_status,
+                          velox_stream_t stream) {
   if (T <= 0 || H <= 0 || W <= 0 || n_chunks <= 0 || b_tok <= 0) return VELOX_ERR_INVALID_ARG;
   if ((long long)n_chunks * T * H * W > kInt32Max) return VELOX_ERR_UNSUPPORTED;
-  if (W < H || (W % 2 == 1 && H % 2 == 0)) return VELOX_ERR_UNSUPPORTED;
+  if (!thw && (W < H || (W % 2 == 1 && H % 2 == 0))) return VELOX_ERR_UNSUPPORTED;
   if (((long long)T * H * W) % b_tok != 0) return VELOX_ERR_UNSUPPORTED;
   if (b_tok > 1024) return VELOX_ERR_UNSUPPORTED;
   const bool want_nbr = nbr_ids != nullptr || nbr_cnt != nullptr;
@@ -115,8 +132,32 @@ velox_status velox_gilbert_order(int T, int H, int W, int n_chunks, int b_tok, i
   if (st != VELOX_OK) return st;
   return from_cuda(velox::launch_gilbert(T, H, W, n_chunks, b_tok, q_chunk, cache_first_block,
                                          n_cache_blocks, rank_of_cell, cell_of_rank,
-                                         block_of_cell, nbr_ids, nbr_cnt, S_max, dev_status,
+                                         block_of_cell, nbr_ids, nbr_cnt, S_max, thw, dev_status,
                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+velox_status velox_gilbert_order(int T, int H, int W, int n_chunks, int b_tok, int q_chunk,
+                                 int cache_first_block, int n_cache_blocks,
+                                 int32_t *rank_of_cell, int32_t *cell_of_rank,
+                                 int32_t *block_of_cell, int32_t *nbr_ids, int32_t *nbr_cnt,
+                                 int S_max, int32_t *dev_status, velox_stream_t stream) {
+  return order_common(T, H, W, n_chunks, b_tok, q_chunk, cache_first_block, n_cache_blocks,
+                      rank_of_cell, cell_of_rank, block_of_cell, nbr_ids, nbr_cnt, S_max, 0,
+                      dev_status, stream);
+}
+
+velox_status velox_thw_linear_order(int T, int H, int W, int n_chunks, int b_tok, int q_chunk,
+                                    int cache_first_block, int n_cache_blocks,
+                                    int32_t *rank_of_cell, int32_t *cell_of_rank,
+                                    int32_t *block_of_cell, int32_t *nbr_ids, int32_t *nbr_cnt,
+                                    int S_max, int32_t *dev_status, velox_stream_t stream) {
+  return order_common(T, H, W, n_chunks, b_tok, q_chunk, cache_first_block, n_cache_blocks,
+                      rank_of_cell, cell_of_rank, block_of_cell, nbr_ids, nbr_cnt, S_max, 1,
+                      dev_status, stream);
 }
 
 velox_status velox_workspace_size(int H, int N, int M, int d, size_t *bytes) {
@@ -196,12 +237,16 @@ velox_status velox_route_schedule(const int32_t *route_len, int rows, int R_max,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
-velox_status velox_block_sparse_attn(const velox_bf16 *Q, const velox_bf16 *K,
-                                     const velox_bf16 *V, const int32_t *route_ids,
-                                     const int32_t *route_len, const int32_t *row_order,
-                                     int R_max, int H, int N, int M,
-                                     int d, int b_tok, float softmax_scale, velox_bf16 *O,
-                                     float *lse, int32_t *dev_status, velox_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+velox_status attn_common(const velox_bf16 *Q, const velox_bf16 *K, const velox_bf16 *V,
+                         const int32_t *route_ids, const int32_t *route_len,
+                         const int32_t *row_order, int R_max, const velox_bf16 *K_cur,
+                         const velox_bf16 *V_cur, int N_cur, int H, int N, int M, int d,
+                         int b_tok, float softmax_scale, velox_bf16 *O, float *lse,
+                         int32_t *dev_status, velox_stream_t stream) {
   if (!Q || !K || !V || !O || H <= 0 || N <= 0 || M <= 0) return VELOX_ERR_INVALID_ARG;
   if (d != VELOX_HEAD_DIM || b_tok != VELOX_BLOCK_TOK) return VELOX_ERR_UNSUPPORTED;
   if (M > VELOX_MAX_BLOCKS || (long long)M * b_tok > kInt32Max ||
@@ -213,6 +258,12 @@ velox_status velox_block_sparse_attn(const velox_bf16 *Q, const velox_bf16 *K,
     if (R_max <= 0) return VELOX_ERR_INVALID_ARG;
     if (R_max > VELOX_MAX_ROUTE) return VELOX_ERR_UNSUPPORTED;
   }
+  if (N_cur < 0) return VELOX_ERR_INVALID_ARG;
+  if (N_cur > 0) {
+    if (!K_cur || !V_cur) return VELOX_ERR_INVALID_ARG;
+    if ((long long)N_cur * b_tok > kInt32Max) return VELOX_ERR_UNSUPPORTED;
+    if (!aligned16(K_cur) || !aligned16(V_cur)) return VELOX_ERR_INVALID_ARG;
+  }
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
     return VELOX_ERR_INVALID_ARG;
   if (std::isnan(softmax_scale) || std::isinf(softmax_scale)) return VELOX_ERR_INVALID_ARG;
@@ -220,12 +271,79 @@ velox_status velox_block_sparse_attn(const velox_bf16 *Q, const velox_bf16 *K,
   velox_status st = check_device();
   if (st != VELOX_OK) return st;
   bool map_failed = false;
-  cudaError_t e = velox::launch_attn(Q, K, V, route_ids, route_len, row_order, R_max, H, N, M,
-                                     scale, O, lse,
-                                     dev_status, reinterpret_cast<cudaStream_t>(stream),
-                                     &map_failed);
+  cudaError_t e = velox::launch_attn(Q, K, V, route_ids, route_len, row_order, R_max,
+                                     N_cur > 0 ? K_cur : nullptr, N_cur > 0 ? V_cur : nullptr,
+                                     N_cur, H, N, M, scale, O, lse, dev_status,
+                                     reinterpret_cast<cudaStream_t>(stream), &map_failed);
   if (map_failed) return VELOX_ERR_CUDA;
   return from_cuda(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+velox_status velox_block_sparse_attn(const velox_bf16 *Q, const velox_bf16 *K,
+                                     const velox_bf16 *V, const int32_t *route_ids,
+                                     const int32_t *route_len, const int32_t *row_order,
+                                     int R_max, int H, int N, int M, int d, int b_tok,
+                                     float softmax_scale, velox_bf16 *O, float *lse,
+                                     int32_t *dev_status, velox_stream_t stream) {
+  return attn_common(Q, K, V, route_ids, route_len, row_order, R_max, nullptr, nullptr, 0, H, N,
+                     M, d, b_tok, softmax_scale, O, lse, dev_status, stream);
+}
+
+velox_status velox_two_phase_attn(const velox_bf16 *Q, const velox_bf16 *K, const velox_bf16 *V,
+                                  const int32_t *route_ids, const int32_t *route_len,
+                                  const int32_t *row_order, int R_max, const velox_bf16 *K_cur,
+                                  const velox_bf16 *V_cur, int N_cur, int H, int N, int M, int d,
+                                  int b_tok, float softmax_scale, velox_bf16 *O, float *lse,
+                                  int32_t *dev_status, velox_stream_t stream) {
+  if (N_cur <= 0 || !K_cur || !V_cur) return VELOX_ERR_INVALID_ARG;
+  return attn_common(Q, K, V, route_ids, route_len, row_order, R_max, K_cur, V_cur, N_cur, H, N,
+                     M, d, b_tok, softmax_scale, O, lse, dev_status, stream);
+}
+
+velox_status velox_slab_overlap(const velox_camera *cams, int n_cams, const velox_slab *q_slabs,
+                                int N, const velox_slab *h_slabs, int M, int grid, float *g,
+                                int32_t *dev_status, velox_stream_t stream) {
+  if (!cams || !q_slabs || !h_slabs || !g || !dev_status) return VELOX_ERR_INVALID_ARG;
+  if (n_cams <= 0 || N <= 0 || M <= 0 || grid < 1) return VELOX_ERR_INVALID_ARG;
+  if (grid > 32 || N > 65535 || (long long)N * M > kInt32Max) return VELOX_ERR_UNSUPPORTED;
+  velox_status st = check_device();
+  if (st != VELOX_OK) return st;
+  return from_cuda(velox::launch_slab_overlap(cams, n_cams, q_slabs, N, h_slabs, M, grid, g,
+                                              dev_status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+velox_status velox_coverage(const velox_camera *cams, int n_cams, const velox_slab *q_slabs,
+                            const float *q_uvz, int N, int b, const velox_slab *h_slabs, int M,
+                            float eta, float *rho, uint8_t *covered, int32_t *dev_status,
+                            velox_stream_t stream) {
+  if (!cams || !q_slabs || !q_uvz || !h_slabs || !rho || !covered || !dev_status)
+    return VELOX_ERR_INVALID_ARG;
+  if (n_cams <= 0 || N <= 0 || M <= 0 || b <= 0 || std::isnan(eta)) return VELOX_ERR_INVALID_ARG;
+  if (b > 128) return VELOX_ERR_UNSUPPORTED;
+  velox_status st = check_device();
+  if (st != VELOX_OK) return st;
+  return from_cuda(velox::launch_coverage(cams, n_cams, q_slabs, q_uvz, N, b, h_slabs, M, eta, rho,
+                                          covered, dev_status,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+velox_status velox_route_audit(const float *p, const float *g, int H, int N, int M,
+                              const velox_route_params *prm, int k_geo, int k_fuse,
+                              int32_t *counts, velox_stream_t stream) {
+  if (!p || !g || !prm || !counts || H <= 0 || N <= 0 || M <= 0) return VELOX_ERR_INVALID_ARG;
+  if (k_geo < 1 || k_fuse < 1) return VELOX_ERR_INVALID_ARG;
+  if (!std::isfinite(prm->lambda) || !std::isfinite(prm->tau) || !std::isfinite(prm->g_ref) ||
+      !(prm->g_ref > 0.f) || !(prm->lambda >= 0.f))
+    return VELOX_ERR_INVALID_ARG;
+  if (M > velox::audit_max_blocks() || (long long)H * N > kInt32Max) return VELOX_ERR_UNSUPPORTED;
+  velox_status st = check_device();
+  if (st != VELOX_OK) return st;
+  return from_cuda(velox::launch_audit(p, g, H, N, M, prm->lambda, prm->tau, prm->g_ref, k_geo,
+                                       k_fuse, counts, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -30,6 +30,11 @@
 //               use the same max.  Epilogue: O / l -> bf16, lse.
 // A pre-pass compacts the route into shared memory, skipping ids outside
 // [0, M) and repeats (flagged in dev_status).
+//
+// Two-phase form (digest, "Reproducibility": the two-phase tile loop): after
+// the routed history tiles the same loop visits the n_cur tiles of the
+// current chunk's own K/V (separate tensors), under the same online softmax,
+// so one normaliser covers both phases.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -67,6 +72,7 @@ struct AttnArgs {
   int R_max;
   int N, M;
   int rows;                  // H * N
+  int n_cur;                 // current-chunk tiles after the routed ones (0: none)
   float scale_log2;  // softmax_scale * log2(e)
   uint16_t *O;
   float *lse;
@@ -106,7 +112,8 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, AttnArgs a) {
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
+                const __grid_constant__ CUtensorMap tmVc, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -200,7 +207,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const int n = *s_nvalid;
+  const int n_hist = *s_nvalid;
+  const int n = n_hist + a.n_cur;  // tiles of both phases
   const uint32_t tmem = *s_tmem;
 
   if (warp == 0) {
@@ -209,6 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
+      if (a.n_cur > 0) {
+        prefetch_tmap(&tmKc);
+        prefetch_tmap(&tmVc);
+      }
       mbar_arrive_expect_tx(q_full, kTileBytes);
       tma_load_3d(sQ, &tmQ, q_full, 0, i * BM, h);
       tma_load_3d(sQ + kHalfBytes, &tmQ, q_full, 64, i * BM, h);
@@ -218,8 +230,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t use = li / nslot;
         if (!mbar_wait(&slot_empty[s], (use & 1) ^ 1, s_abort)) break;
         const int j = li >> 1;
-        const int tile = dense ? j : tiles[j];
-        const CUtensorMap *map = (li & 1) ? &tmV : &tmK;
+        const bool hist = j < n_hist;
+        const int tile = hist ? (dense ? j : tiles[j]) : j - n_hist;
+        const CUtensorMap *map = (li & 1) ? (hist ? &tmV : &tmVc) : (hist ? &tmK : &tmKc);
         uint8_t *dst = ring + s * kTileBytes;
         mbar_arrive_expect_tx(&slot_full[s], kTileBytes);
         tma_load_3d(dst, map, &slot_full[s], 0, tile * BN, h);
@@ -440,13 +453,17 @@ int attn_max_route() { return kMaxRoute; }
 
 cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                         const int32_t *route_ids, const int32_t *route_len,
-                        const int32_t *row_order, int R_max, int H,
-                        int N, int M, float softmax_scale, uint16_t *O, float *lse,
-                        int32_t *dev_status, cudaStream_t stream, bool *map_failed) {
+                        const int32_t *row_order, int R_max, const uint16_t *K_cur,
+                        const uint16_t *V_cur, int N_cur, int H, int N, int M,
+                        float softmax_scale, uint16_t *O, float *lse, int32_t *dev_status,
+                        cudaStream_t stream, bool *map_failed) {
   *map_failed = false;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mkc, mvc;
+  const bool cur = K_cur != nullptr && N_cur > 0;
   if (!make_map(&mq, Q, N * BM, H) || !make_map(&mk, K, M * BN, H) ||
-      !make_map(&mv, V, M * BN, H)) {
+      !make_map(&mv, V, M * BN, H) ||
+      !make_map(&mkc, cur ? K_cur : K, cur ? N_cur * BN : M * BN, H) ||
+      !make_map(&mvc, cur ? V_cur : V, cur ? N_cur * BN : M * BN, H)) {
     *map_failed = true;
     return cudaErrorInvalidValue;
   }
@@ -458,6 +475,7 @@ cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
   a.N = N;
   a.M = M;
   a.rows = H * N;
+  a.n_cur = cur ? N_cur : 0;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.O = O;
   a.lse = lse;
@@ -477,7 +495,7 @@ cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
   cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  attn_kernel<<<H * N, kThreads, smem, stream>>>(mq, mk, mv, a);
+  attn_kernel<<<H * N, kThreads, smem, stream>>>(mq, mk, mv, mkc, mvc, a);
   return cudaGetLastError();
 }
 

@@ -9,7 +9,7 @@ and the smoke run) receive their inputs from here.
 """
 
 from .configs import CONFIGS, Workload, RouteParams, sweep_workload, config
-from .generate import make_inputs, Inputs
+from .generate import make_inputs, make_current, Inputs
 
 __all__ = ["CONFIGS", "Workload", "RouteParams", "sweep_workload", "config",
-           "make_inputs", "Inputs"]
+           "make_inputs", "make_current", "Inputs"]

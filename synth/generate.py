@@ -85,3 +85,14 @@ def make_inputs(wl: Workload, device="cpu", out: Optional[Inputs] = None) -> Inp
     ref = torch.zeros(0, dtype=torch.int32)
     return Inputs(wl=wl, Q=Q, K=K, V=V, g=g.to(device), covered=covered.to(device),
                   ref_ids=ref.to(device))
+
+
+def make_current(wl: Workload, device="cpu"):
+    """K and V of the chunk being generated, [H][N*b][d] bf16 ~ N(0, 1): the
+    second phase of two-phase attention (its own seed, disjoint from Q/K/V)."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device).manual_seed(wl.seed * 7 + 5)
+    shape = (wl.heads, wl.n_q_blocks * wl.b, wl.d)
+    Kc = torch.empty(shape, dtype=torch.bfloat16, device=device).normal_(generator=gen)
+    Vc = torch.empty(shape, dtype=torch.bfloat16, device=device).normal_(generator=gen)
+    return Kc, Vc
