@@ -433,6 +433,80 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
+def _time_us(fn, reps=50, warm=3):
+    for _ in range(warm):
+        fn()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps * 1e3
+
+
+def run_geometry(args):
+    """Slab overlap g and coverage rho at the chunk-48 shape (48 query blocks,
+    2256 history blocks, 8^3 samples per pair, 128 tokens per block): one JSON
+    line with the per-call times.  Not the bench line."""
+    import numpy as np
+    import routed_block_sparse_b200 as rbs
+    from synth.geometry import make_scene, pack_slabs
+
+    N, M, G, b = 48, 2256, 8, 128
+    s = make_scene(20261203, N, M, b)
+    cams = torch.from_numpy(s.cams).cuda()
+    qs = torch.from_numpy(pack_slabs(s.q_slab, s.q_cam)).cuda()
+    hs = torch.from_numpy(pack_slabs(s.h_slab, s.h_cam, s.h_valid)).cuda()
+    uvz = torch.from_numpy(np.ascontiguousarray(s.q_uvz)).cuda()
+    g = torch.empty(N, M, device="cuda")
+    rho = torch.empty(N, device="cuda")
+    cov = torch.empty(N, dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    n_cam = cams.shape[0]
+    t_g = _time_us(lambda: rbs.velox_slab_overlap(cams, n_cam, qs, N, hs, M, G, g, st))
+    t_c = _time_us(lambda: rbs.velox_coverage(cams, n_cam, qs, uvz, N, b, hs, M, 0.9, rho, cov,
+                                              st))
+    nz = int((g > 0).sum().item())
+    print(json.dumps({"geometry": "chunk48", "N": N, "M": M, "grid": G, "b": b,
+                      "slab_overlap_us": t_g, "coverage_us": t_c,
+                      "pairs_per_s": N * M / (t_g * 1e-6), "nonzero_pairs": nz,
+                      "covered_blocks": int(cov.sum().item()),
+                      "dev_status": int(st.item())}), flush=True)
+
+
+def run_two_phase(args):
+    """Routed history tiles plus the 48 blocks of the current chunk (chunk-48
+    shape): the one-pass two-phase kernel against the history-only routed
+    call.  One JSON line.  Not the bench line."""
+    import routed_block_sparse_b200 as rbs
+    from routed_block_sparse_b200.pipeline import layer_for
+    from synth import config, make_current, make_inputs
+
+    wl = config(3, 0)
+    inp = make_inputs(wl, "cuda")
+    Kc, Vc = make_current(wl, "cuda")
+    layer = layer_for(wl)
+    layer.forward(inp.Q, inp.K, inp.V, inp.g, inp.covered)
+    torch.cuda.synchronize()
+    H, N, M = wl.heads, wl.n_q_blocks, wl.n_kv_blocks
+    hist = float(layer.route_len.sum().item())
+    t_r = _time_us(lambda: layer.attend(inp.Q, inp.K, inp.V), reps=20)
+
+    def two():
+        rbs.velox_two_phase_attn(inp.Q, inp.K, inp.V, layer.route_ids, layer.route_len,
+                                 layer.R_max, Kc, Vc, N, H, N, M, 128, 128, layer.softmax_scale,
+                                 layer.O, layer.lse, layer.dev_status, row_order=layer.row_order)
+    t_2 = _time_us(two, reps=20)
+    tiles = hist + H * N * N
+    print(json.dumps({"two_phase": "chunk48", "mean_route_len": hist / (H * N),
+                      "current_blocks": N, "routed_us": t_r, "two_phase_us": t_2,
+                      "two_phase_tflops": 4.0 * 128 ** 3 * tiles / (t_2 * 1e-6) / 1e12,
+                      "routed_tflops": 4.0 * 128 ** 3 * hist / (t_r * 1e-6) / 1e12,
+                      "dev_status": layer.status()}), flush=True)
+
+
 def run_layers(args):
     """Full denoising step at chunk 48: `args.layers` layers with independent
     per-layer inputs (seeded per layer), regenerated into reused buffers
@@ -490,6 +564,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="history-length sweep: routed vs dense attention per M (extra lines)")
+    ap.add_argument("--geometry", action="store_true",
+                    help="time slab overlap and coverage at the chunk-48 shape")
+    ap.add_argument("--two-phase", action="store_true",
+                    help="time two-phase attention (history routes + current chunk)")
     ap.add_argument("--layers", type=int, default=0,
                     help="full-step mode: this many chunk-48 layers with per-layer inputs "
                          "(extra line with the summed route-build and attention times)")
@@ -507,6 +585,12 @@ def main():
     try:
         if args.sweep:
             run_sweep(args)
+            return
+        if args.geometry:
+            run_geometry(args)
+            return
+        if args.two_phase:
+            run_two_phase(args)
             return
         if args.layers:
             run_layers(args)
