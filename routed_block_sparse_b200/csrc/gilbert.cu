@@ -111,11 +111,15 @@ __device__ void frame_cell(int W, int H, int k, int &cx, int &cy) {
 
 struct Lattice {
   int T, H, W, n_chunks, b;
+  int thw;  // 1: THW-linear (raster) order instead of the global Gilbert order
   __device__ int HW() const { return H * W; }
+  __device__ bool mirrored(int f) const { return !thw && (f & 1); }
+  // position of in-frame cell (x, y) on the frame's walk
+  __device__ int in_frame(int x, int y) const { return thw ? y * W + x : frame_rank(W, H, x, y); }
   // global rank of cell (f, y, x)
   __device__ int rank(int f, int y, int x) const {
-    int xm = (f & 1) ? (W - 1 - x) : x;
-    return f * H * W + frame_rank(W, H, xm, y);
+    int xm = mirrored(f) ? (W - 1 - x) : x;
+    return f * H * W + in_frame(xm, y);
   }
 };
 
@@ -166,7 +170,7 @@ __global__ void neighbour_kernel(Lattice L, int q_chunk, int cache_first, int n_
   if (use_table) {
     for (int cidx = threadIdx.x; cidx < HW; cidx += blockDim.x) {
       const int y = cidx / L.W, x = cidx - y * L.W;
-      const int rk = frame_rank(L.W, L.H, x, y);
+      const int rk = L.in_frame(x, y);
       r2[cidx] = rk;
       inv[rk] = cidx;
     }
@@ -184,14 +188,17 @@ __global__ void neighbour_kernel(Lattice L, int q_chunk, int cache_first, int n_
       const int cidx = inv[k];
       y = cidx / L.W;
       xm = cidx - y * L.W;
+    } else if (L.thw) {
+      y = k / L.W;
+      xm = k - y * L.W;
     } else {
       frame_cell(L.W, L.H, k, xm, y);
     }
-    const int x = (f & 1) ? (L.W - 1 - xm) : xm;
+    const int x = L.mirrored(f) ? (L.W - 1 - xm) : xm;
     const int f2 = f + o / 9 - 1, y2 = y + (o / 3) % 3 - 1, x2 = x + o % 3 - 1;
     if (f2 < 0 || f2 >= F || y2 < 0 || y2 >= L.H || x2 < 0 || x2 >= L.W) continue;
-    const int xm2 = (f2 & 1) ? (L.W - 1 - x2) : x2;
-    const int r2v = use_table ? r2[y2 * L.W + xm2] : frame_rank(L.W, L.H, xm2, y2);
+    const int xm2 = L.mirrored(f2) ? (L.W - 1 - x2) : x2;
+    const int r2v = use_table ? r2[y2 * L.W + xm2] : L.in_frame(xm2, y2);
     const int u = (int)(((long long)f2 * HW + r2v) / L.b);
     if (u == qb || u < cache_first || u >= cache_first + n_cache) continue;
     const int bit = u - wlo;  // within the window by construction
@@ -235,9 +242,9 @@ __global__ void neighbour_kernel(Lattice L, int q_chunk, int cache_first, int n_
 cudaError_t launch_gilbert(int T, int H, int W, int n_chunks, int b, int q_chunk,
                            int cache_first, int n_cache, int32_t *rank_of_cell,
                            int32_t *cell_of_rank, int32_t *block_of_cell, int32_t *nbr_ids,
-                           int32_t *nbr_cnt, int S_max, int32_t *dev_status,
+                           int32_t *nbr_cnt, int S_max, int thw, int32_t *dev_status,
                            cudaStream_t stream) {
-  Lattice L{T, H, W, n_chunks, b};
+  Lattice L{T, H, W, n_chunks, b, thw};
   const int n_cells = n_chunks * T * H * W;
   if (rank_of_cell || cell_of_rank || block_of_cell) {
     int grid = (n_cells + 255) / 256;

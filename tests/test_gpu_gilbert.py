@@ -93,3 +93,48 @@ def test_unsupported_lattices_raise(lib):
         lib.velox_gilbert_order(2, 2, 3, 1, 3, rank_of_cell=out)   # W odd, H even
     with pytest.raises(lib.VeloxError):
         lib.velox_gilbert_order(3, 3, 4, 1, 5, rank_of_cell=out)   # 36 % 5 != 0
+
+
+THW_CASES = [
+    # T, H, W, b, n_chunks
+    (3, 3, 4, 2, 2),          # the pages' toy lattice
+    (4, 32, 48, 128, 48),     # chunk-48 rollout lattice
+    (2, 8, 5, 8, 3),          # W < H (allowed for a raster order)
+]
+
+
+@pytest.mark.parametrize("T,H,W,b,nc", THW_CASES)
+def test_thw_order_bit_exact(lib, T, H, W, b, nc):
+    n = nc * T * H * W
+    rank = torch.full((n,), -7, dtype=torch.int32, device="cuda")
+    block = torch.full((n,), -7, dtype=torch.int32, device="cuda")
+    lib.velox_thw_linear_order(T, H, W, nc, b, rank_of_cell=rank, block_of_cell=block)
+    torch.cuda.synchronize()
+    r_ref, _, b_ref = gilbert.thw_linear_order(T, H, W, nc, b)
+    assert np.array_equal(rank.cpu().numpy(), r_ref)
+    assert np.array_equal(block.cpu().numpy(), b_ref)
+
+
+@pytest.mark.parametrize("T,H,W,b,nc,qc,first,M", [
+    (3, 3, 4, 2, 2, 1, 0, 18),
+    (4, 32, 48, 128, 48, 47, 0, 2256),  # chunk-48
+    (2, 8, 5, 8, 3, 1, 2, 12),
+    (1, 96, 96, 128, 3, 2, 0, 144),     # frame above the shared-memory table size
+])
+def test_thw_neighbours_bit_exact(lib, T, H, W, b, nc, qc, first, M):
+    N = T * H * W // b
+    S_max = 64
+    ids = torch.full((N, S_max), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.full((N,), -7, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lib.velox_thw_linear_order(T, H, W, nc, b, qc, first, M, nbr_ids=ids, nbr_cnt=cnt,
+                               S_max=S_max, dev_status=st)
+    torch.cuda.synchronize()
+    ref = gilbert.neighbour_blocks(T, H, W, nc, b, qc, first, M, layout="thw")
+    assert int(st.item()) == 0
+    c = cnt.cpu().numpy()
+    got = ids.cpu().numpy()
+    for i in range(N):
+        assert c[i] == len(ref[i])
+        assert got[i, :c[i]].tolist() == ref[i]
+        assert np.all(got[i, c[i]:] == -1)
