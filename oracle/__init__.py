@@ -38,9 +38,14 @@ Modules and the passages they follow:
                  page, "03 · Results"; digest, results table; onedev.kr
                  summary, "Results").
 
+- ``slabs``      the slab-table build (token rectangle and 10/90 percentile
+                 depth interval per history block) and the recency-priority
+                 multiwarp query depth (digest, "Method steps", Eq. 4-6;
+                 project page, "02 · Method", steps 01-02).
+
 Every function here is pinned by the ``-m "not gpu"`` tests in
 ``tests/test_oracle_*.py`` against invariants, closed forms, textbook routines
 and brute force, not against itself.
 """
 
-from . import gilbert, importance, route, attention, geometry, audit  # noqa: F401
+from . import gilbert, importance, route, attention, geometry, audit, slabs  # noqa: F401
