@@ -447,33 +447,77 @@ def _time_us(fn, reps=50, warm=3):
 
 
 def run_geometry(args):
-    """Slab overlap g and coverage rho at the chunk-48 shape (48 query blocks,
-    2256 history blocks, 8^3 samples per pair, 128 tokens per block): one JSON
-    line with the per-call times.  Not the bench line."""
+    """The geometry chain at the chunk-48 shape, one JSON line of per-call
+    times (not the bench line): slab table of the 2256 history blocks (188
+    frames of 32 x 48 tokens, 2 x 2 depth samples per token), multiwarp depth
+    of the 4 current frames from the first and last frames of the 30 most
+    recent chunks, the current chunk's 48 query slabs and tokens, slab
+    overlap g (8^3 samples per pair) and coverage rho."""
     import numpy as np
     import routed_block_sparse_b200 as rbs
-    from synth.geometry import make_scene, pack_slabs
+    from synth.depth import make_rollout
 
-    N, M, G, b = 48, 2256, 8, 128
-    s = make_scene(20261203, N, M, b)
-    cams = torch.from_numpy(s.cams).cuda()
-    qs = torch.from_numpy(pack_slabs(s.q_slab, s.q_cam)).cuda()
-    hs = torch.from_numpy(pack_slabs(s.h_slab, s.h_cam, s.h_valid)).cuda()
-    uvz = torch.from_numpy(np.ascontiguousarray(s.q_uvz)).cuda()
+    T, H, W, b, nc, s = 4, 32, 48, 128, 48, 2
+    q_chunk = nc - 1
+    per_chunk = T * H * W // b
+    M, N = q_chunk * per_chunk, per_chunk
+    hist_frames = q_chunk * T
+    roll = make_rollout(20261203, nc * T, H, W, s)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    cams = dev(roll.cams)
+    n_cam = cams.shape[0]
+    depth, conf, mask = dev(roll.depth[:hist_frames]), dev(roll.conf[:hist_frames]), \
+        dev(roll.mask[:hist_frames])
+    cell = torch.empty(nc * T * H * W, dtype=torch.int32, device="cuda")
+    rbs.velox_gilbert_order(T, H, W, nc, b, cell_of_rank=cell)
+    src = []
+    for c in range(q_chunk - 1, q_chunk - 31, -1):          # 30 most recent chunks
+        src += [c * T + T - 1, c * T]                        # last, first frame
+    src_depth = dev(roll.depth[src])
+    src_cam = torch.tensor(src, dtype=torch.int32, device="cuda")
+    tgt_cam = torch.arange(hist_frames, hist_frames + T, dtype=torch.int32, device="cuda")
+    hs = torch.empty(M, 8, dtype=torch.int32, device="cuda")
+    qs = torch.empty(N, 8, dtype=torch.int32, device="cuda")
+    zq = torch.empty(T, H, W, device="cuda")
+    uvz = torch.empty(N, b, 3, device="cuda")
     g = torch.empty(N, M, device="cuda")
     rho = torch.empty(N, device="cuda")
     cov = torch.empty(N, dtype=torch.uint8, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    n_cam = cams.shape[0]
-    t_g = _time_us(lambda: rbs.velox_slab_overlap(cams, n_cam, qs, N, hs, M, G, g, st))
-    t_c = _time_us(lambda: rbs.velox_coverage(cams, n_cam, qs, uvz, N, b, hs, M, 0.9, rho, cov,
-                                              st))
-    nz = int((g > 0).sum().item())
-    print(json.dumps({"geometry": "chunk48", "N": N, "M": M, "grid": G, "b": b,
-                      "slab_overlap_us": t_g, "coverage_us": t_c,
-                      "pairs_per_s": N * M / (t_g * 1e-6), "nonzero_pairs": nz,
-                      "covered_blocks": int(cov.sum().item()),
-                      "dev_status": int(st.item())}), flush=True)
+
+    def table():
+        rbs.velox_slab_table(depth, conf, mask, hist_frames, 0, H, W, s, cell, cell.numel(), b, 0,
+                             M, 0.5, 16, 0.1, 0.9, hs, st)
+
+    def warp():
+        rbs.velox_multiwarp(cams, n_cam, src_depth, src_cam, len(src), tgt_cam, T, H, W, s, 2, zq,
+                            st)
+
+    def qtable():
+        rbs.velox_slab_table(zq, None, None, T, hist_frames, H, W, 1, cell, cell.numel(), b,
+                             q_chunk * per_chunk, N, 0.5, 8, 0.1, 0.9, qs, st, token_uvz=uvz)
+
+    def overlap():
+        rbs.velox_slab_overlap(cams, n_cam, qs, N, hs, M, 8, g, st)
+
+    def coverage():
+        rbs.velox_coverage(cams, n_cam, qs, uvz, N, b, hs, M, 0.9, rho, cov, st)
+
+    out = {"geometry": "chunk48", "N": N, "M": M, "grid": 8, "b": b, "depth_samples": s,
+           "multiwarp_sources": len(src)}
+    for name, fn in (("slab_table", table), ("multiwarp", warp), ("query_slabs", qtable),
+                     ("slab_overlap", overlap), ("coverage", coverage)):
+        out[name + "_us"] = _time_us(fn)
+
+    def chain():
+        table(); warp(); qtable(); overlap(); coverage()
+    out["chain_us"] = _time_us(chain, reps=20)
+    torch.cuda.synchronize()
+    out.update({"valid_history_slabs": int(hs[:, 7].sum().item()),
+                "query_holes": float((zq == 0).float().mean().item()),
+                "nonzero_pairs": int((g > 0).sum().item()),
+                "covered_blocks": int(cov.sum().item()), "dev_status": int(st.item())})
+    print(json.dumps(out), flush=True)
 
 
 def run_two_phase(args):

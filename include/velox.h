@@ -82,7 +82,8 @@ typedef enum {
 #define VELOX_DEV_WAIT_TIMEOUT   0x20  /* bounded mbarrier wait gave up        */
 #define VELOX_DEV_ROUTE_CAPACITY 0x40  /* route row longer than R_max: cut     */
 #define VELOX_DEV_BAD_ROW_ORDER  0x80  /* row_order entry outside [0, H*N)      */
-#define VELOX_DEV_BAD_CAMERA     0x100 /* slab camera index outside [0, n_cams)  */
+#define VELOX_DEV_BAD_CAMERA     0x100 /* camera index outside [0, n_cams)       */
+#define VELOX_DEV_BAD_CELL       0x200 /* block cell outside the lattice / frames  */
 
 /* Supported sizes of the importance and attention calls. */
 #define VELOX_HEAD_DIM   128
@@ -431,6 +432,66 @@ VELOX_API velox_status velox_coverage(const velox_camera *cams, int n_cams,
 VELOX_API velox_status velox_route_audit(const float *p, const float *g, int H, int N, int M,
                                          const velox_route_params *prm, int k_geo, int k_fuse,
                                          int32_t *counts, velox_stream_t stream);
+
+/*
+ * velox_slab_table -- the frustum slab of every history block from depth.
+ *
+ * Defined by: digest, "Method steps", step one (Eq. 4-5: reliable depth
+ * back-projected and bucketed by Gilbert block, 10/90 percentile depth
+ * interval per block) and "Prerequisites" (a slab is a token rectangle plus
+ * a depth interval); project page, "02 · Method", step 01.
+ *
+ * depth, conf [F][H s][W s] fp32 and mask [F][H s][W s] uint8 (conf and
+ * mask nullable) hold global frames frame_base .. frame_base + F - 1, s x s
+ * samples per token.  cell_of_rank [n_cells] is a token order (from
+ * velox_gilbert_order or velox_thw_linear_order); block r covers ranks
+ * r b_tok .. r b_tok + b_tok - 1.  For r = first_block + j, j < n_blocks:
+ * slabs[j] = {u0, u1, v0, v1} = the bounding box [min x, max x + 1) x
+ * [min y, max y + 1) of its cells, {zlo, zhi} = percentiles p_lo and p_hi
+ * (linear interpolation between order statistics at (n - 1) p, fp64, rounded
+ * to fp32) of its reliable samples (mask set, conf >= c_min, 0 < depth <
+ * inf), cam = its global frame, valid = (n >= n_min); an invalid slab is all
+ * zeros.  A block whose cells leave the lattice, straddle frames or lie
+ * outside the given frames flags VELOX_DEV_BAD_CELL and is invalid.
+ * token_uvz (nullable; only with s == 1) [n_blocks][b_tok][3]: the tokens of
+ * each block in rank order as (x + 0.5, y + 0.5, depth), depth 0 where the
+ * sample is not reliable -- the per-token input of velox_coverage when the
+ * depth is a query frame's multiwarp depth.
+ * Requires H W % b_tok == 0, 1 <= s, b_tok s^2 <= 16384.
+ */
+VELOX_API velox_status velox_slab_table(const float *depth, const float *conf,
+                                        const uint8_t *mask, int F, int frame_base, int H, int W,
+                                        int s, const int32_t *cell_of_rank, int n_cells,
+                                        int b_tok, int first_block, int n_blocks, float c_min,
+                                        int n_min, double p_lo, double p_hi, velox_slab *slabs,
+                                        float *token_uvz, int32_t *dev_status,
+                                        velox_stream_t stream);
+
+/*
+ * velox_multiwarp -- recency-priority multiwarp depth z^Q of target frames.
+ *
+ * Defined by: digest, "Method steps", step two (Eq. 6: first and last frame
+ * depths of the K = 30 most recent reconstructed chunks forward-warped to the
+ * target camera; each token takes the median of the newest frame that gives
+ * it at least k_warp = 2 samples) and "Recency-priority multiwarp".
+ *
+ * src_depth [S][H s][W s] fp32 with cameras src_cam [S] (device), newest
+ * first; tgt_cam [n_tgt] (device).  Every source sample (px, py) with depth
+ * z > 0 sits at token coordinates ((px + 0.5) / s, (py + 0.5) / s); it is
+ * back-projected with its camera and projected into the target camera; it
+ * lands in target token (floor u', floor v') when its target depth is > 0
+ * and 0 <= u' < W, 0 <= v' < H, with that depth as its value.
+ * zq [n_tgt][H][W] fp32: the median (mean of the two middle values for an
+ * even count, fp64 rounded to fp32) of the first source, newest first, that
+ * gives the token >= k_warp samples; 0 (a hole) if none does.  A camera index
+ * out of range flags VELOX_DEV_BAD_CAMERA and that source (target) is
+ * skipped (left 0).  Requires H W s^2 <= 32768.
+ */
+VELOX_API velox_status velox_multiwarp(const velox_camera *cams, int n_cams,
+                                       const float *src_depth, const int32_t *src_cam, int S,
+                                       const int32_t *tgt_cam, int n_tgt, int H, int W, int s,
+                                       int k_warp, float *zq, int32_t *dev_status,
+                                       velox_stream_t stream);
 
 #ifdef __cplusplus
 }

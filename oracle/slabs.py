@@ -117,6 +117,25 @@ def slab_table(depth, conf, mask, cell_of_rank, H: int, W: int, b: int, frame_ba
     return slab, cam, valid
 
 
+def block_tokens(depth, conf, mask, cell_of_rank, H: int, W: int, b: int, frame_base: int,
+                 first_block: int, n_blocks: int, c_min: float = 0.5) -> np.ndarray:
+    """[n][b][3]: the tokens of each block in rank order as (x + 0.5, y + 0.5,
+    depth), depth 0 where it is not a reliable sample (s = 1): the per-token
+    input of the coverage when depth is a multiwarp map."""
+    HW = H * W
+    out = np.zeros((n_blocks, b, 3), dtype=np.float32)
+    for j in range(n_blocks):
+        for t in range(b):
+            c = int(cell_of_rank[(first_block + j) * b + t])
+            f, rem = divmod(c, HW)
+            y, x = divmod(rem, W)
+            z = float(depth[f - frame_base, y, x])
+            ok = z > 0.0 and math.isfinite(z) and (mask is None or mask[f - frame_base, y, x] != 0)
+            ok = ok and (conf is None or float(conf[f - frame_base, y, x]) >= float(F(c_min)))
+            out[j, t] = [x + 0.5, y + 0.5, z if ok else 0.0]
+    return out
+
+
 def warp_sample(cam_src, cam_tgt, u, v, z, H: int, W: int):
     """Target token (x, y) and target depth of source point (u, v) at depth z,
     or None when it does not land in the target frame."""

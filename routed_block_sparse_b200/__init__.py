@@ -31,6 +31,7 @@ DEV_WAIT_TIMEOUT = 0x20
 DEV_ROUTE_CAPACITY = 0x40
 DEV_BAD_ROW_ORDER = 0x80
 DEV_BAD_CAMERA = 0x100
+DEV_BAD_CELL = 0x200
 HEAD_DIM = 128
 BLOCK_TOK = 128
 MAX_BLOCKS = 65536
@@ -41,7 +42,8 @@ EXPORTS = ("velox_status_string", "velox_abi_version", "velox_gilbert_order",
            "velox_workspace_size", "velox_block_importance", "velox_route_build",
            "velox_block_sparse_attn", "velox_block_importance_noalloc",
            "velox_route_schedule", "velox_two_phase_attn", "velox_slab_overlap",
-           "velox_coverage", "velox_route_audit", "velox_thw_linear_order")
+           "velox_coverage", "velox_route_audit", "velox_thw_linear_order",
+           "velox_slab_table", "velox_multiwarp")
 
 
 class VeloxError(RuntimeError):
@@ -90,6 +92,12 @@ def _load() -> ctypes.CDLL:
     lib.velox_coverage.argtypes = [P, I, P, P, I, I, P, I, F, P, P, P, P]
     lib.velox_route_audit.restype = I
     lib.velox_route_audit.argtypes = [P, P, I, I, I, ctypes.POINTER(RouteParams), I, I, P, P]
+    D = ctypes.c_double
+    lib.velox_slab_table.restype = I
+    lib.velox_slab_table.argtypes = [P, P, P, I, I, I, I, I, P, I, I, I, I, F, I, D, D, P, P, P,
+                                     P]
+    lib.velox_multiwarp.restype = I
+    lib.velox_multiwarp.argtypes = [P, I, P, P, I, P, I, I, I, I, I, P, P, P]
     lib.velox_two_phase_attn.restype = I
     lib.velox_two_phase_attn.argtypes = [P, P, P, P, P, P, I, P, P, I, I, I, I, I, I, F, P, P, P,
                                          P]
@@ -231,3 +239,21 @@ def velox_route_audit(p, g, H, N, M, prm, k_geo, k_fuse, counts, stream=None):
     st = _lib.velox_route_audit(_ptr(p), _ptr(g), H, N, M, ctypes.byref(prm), k_geo, k_fuse,
                                 _ptr(counts), _stream(stream))
     _check("velox_route_audit", st)
+
+
+def velox_slab_table(depth, conf, mask, F, frame_base, H, W, s, cell_of_rank, n_cells, b_tok,
+                     first_block, n_blocks, c_min, n_min, p_lo, p_hi, slabs, dev_status,
+                     token_uvz=None, stream=None):
+    st = _lib.velox_slab_table(_ptr(depth), _ptr(conf), _ptr(mask), F, frame_base, H, W, s,
+                               _ptr(cell_of_rank), n_cells, b_tok, first_block, n_blocks,
+                               float(c_min), n_min, float(p_lo), float(p_hi), _ptr(slabs),
+                               _ptr(token_uvz), _ptr(dev_status), _stream(stream))
+    _check("velox_slab_table", st)
+
+
+def velox_multiwarp(cams, n_cams, src_depth, src_cam, S, tgt_cam, n_tgt, H, W, s, k_warp, zq,
+                    dev_status, stream=None):
+    st = _lib.velox_multiwarp(_ptr(cams), n_cams, _ptr(src_depth), _ptr(src_cam), S,
+                              _ptr(tgt_cam), n_tgt, H, W, s, k_warp, _ptr(zq), _ptr(dev_status),
+                              _stream(stream))
+    _check("velox_multiwarp", st)

@@ -40,6 +40,17 @@ cudaError_t launch_coverage(const velox_camera *cams, int n_cams, const velox_sl
                             float eta, float *rho, uint8_t *covered, int32_t *dev_status,
                             cudaStream_t stream);
 int audit_max_blocks();
+int multiwarp_max_samples();
+int slab_table_max_samples();
+cudaError_t launch_slab_table(const float *depth, const float *conf, const uint8_t *mask, int F,
+                              int frame_base, int H, int W, int s, const int32_t *cell_of_rank,
+                              int n_cells, int b, int first_block, int n_blocks, float c_min,
+                              int n_min, double p_lo, double p_hi, velox_slab *slabs,
+                              float *token_uvz, int32_t *dev_status, cudaStream_t stream);
+cudaError_t launch_multiwarp(const velox_camera *cams, int n_cams, const float *src_depth,
+                             const int32_t *src_cam, int S, const int32_t *tgt_cam, int n_tgt,
+                             int H, int W, int s, int k_warp, float *zq, int32_t *dev_status,
+                             cudaStream_t stream);
 cudaError_t launch_audit(const float *p, const float *g, int H, int N, int M, double lam,
                          double tau, double g_ref, int k_geo, int k_fuse, int32_t *counts,
                          cudaStream_t stream);
@@ -344,6 +355,48 @@ velox_status velox_route_audit(const float *p, const float *g, int H, int N, int
   if (st != VELOX_OK) return st;
   return from_cuda(velox::launch_audit(p, g, H, N, M, prm->lambda, prm->tau, prm->g_ref, k_geo,
                                        k_fuse, counts, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+velox_status velox_slab_table(const float *depth, const float *conf, const uint8_t *mask, int F,
+                             int frame_base, int H, int W, int s, const int32_t *cell_of_rank,
+                             int n_cells, int b_tok, int first_block, int n_blocks, float c_min,
+                             int n_min, double p_lo, double p_hi, velox_slab *slabs,
+                             float *token_uvz, int32_t *dev_status, velox_stream_t stream) {
+  if (!depth || !cell_of_rank || !slabs || !dev_status) return VELOX_ERR_INVALID_ARG;
+  if (token_uvz && s != 1) return VELOX_ERR_UNSUPPORTED;
+  if (F <= 0 || H <= 0 || W <= 0 || s <= 0 || b_tok <= 0 || n_blocks <= 0 || first_block < 0 ||
+      n_cells <= 0 || n_min < 0)
+    return VELOX_ERR_INVALID_ARG;
+  if (!(p_lo >= 0.0 && p_lo <= 1.0 && p_hi >= 0.0 && p_hi <= 1.0) || std::isnan(c_min))
+    return VELOX_ERR_INVALID_ARG;
+  if ((long long)(first_block + (long long)n_blocks) * b_tok > n_cells) return VELOX_ERR_INVALID_ARG;
+  if (((long long)H * W) % b_tok != 0) return VELOX_ERR_UNSUPPORTED;
+  if ((long long)b_tok * s * s > velox::slab_table_max_samples()) return VELOX_ERR_UNSUPPORTED;
+  if ((long long)F * H * W * s * s > kInt32Max || n_blocks > kInt32Max / 2)
+    return VELOX_ERR_UNSUPPORTED;
+  velox_status st = check_device();
+  if (st != VELOX_OK) return st;
+  return from_cuda(velox::launch_slab_table(depth, conf, mask, F, frame_base, H, W, s,
+                                            cell_of_rank, n_cells, b_tok, first_block, n_blocks,
+                                            c_min, n_min, p_lo, p_hi, slabs, token_uvz, dev_status,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+velox_status velox_multiwarp(const velox_camera *cams, int n_cams, const float *src_depth,
+                             const int32_t *src_cam, int S, const int32_t *tgt_cam, int n_tgt,
+                             int H, int W, int s, int k_warp, float *zq, int32_t *dev_status,
+                             velox_stream_t stream) {
+  if (!cams || !src_depth || !src_cam || !tgt_cam || !zq || !dev_status)
+    return VELOX_ERR_INVALID_ARG;
+  if (n_cams <= 0 || S <= 0 || n_tgt <= 0 || H <= 0 || W <= 0 || s <= 0 || k_warp < 1)
+    return VELOX_ERR_INVALID_ARG;
+  if ((long long)H * W * s * s > velox::multiwarp_max_samples() || n_tgt > 65535)
+    return VELOX_ERR_UNSUPPORTED;
+  velox_status st = check_device();
+  if (st != VELOX_OK) return st;
+  return from_cuda(velox::launch_multiwarp(cams, n_cams, src_depth, src_cam, S, tgt_cam, n_tgt, H,
+                                           W, s, k_warp, zq, dev_status,
+                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"
