@@ -484,6 +484,8 @@ def run_geometry(args):
     rho = torch.empty(N, device="cuda")
     cov = torch.empty(N, dtype=torch.uint8, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    mw_ws = torch.empty(rbs.velox_multiwarp_workspace_size(len(src), T, H, W), dtype=torch.uint8,
+                        device="cuda")
 
     def table():
         rbs.velox_slab_table(depth, conf, mask, hist_frames, 0, H, W, s, cell, cell.numel(), b, 0,
@@ -491,7 +493,7 @@ def run_geometry(args):
 
     def warp():
         rbs.velox_multiwarp(cams, n_cam, src_depth, src_cam, len(src), tgt_cam, T, H, W, s, 2, zq,
-                            st)
+                            mw_ws, st)
 
     def qtable():
         rbs.velox_slab_table(zq, None, None, T, hist_frames, H, W, 1, cell, cell.numel(), b,
@@ -551,6 +553,66 @@ def run_two_phase(args):
                       "dev_status": layer.status()}), flush=True)
 
 
+def run_variants(args):
+    """The comparison rows, one JSON line each (not the bench line):
+    the geometry-model audit at the audit scale (config 2), the model-only
+    route (lambda = 0) against the fused route at the chunk-48 shape, and the
+    THW-linear order's neighbour table against the Gilbert order's."""
+    import routed_block_sparse_b200 as rbs
+    from routed_block_sparse_b200.pipeline import audit_metrics, layer_for
+    from synth import config, make_inputs
+
+    # 1. audit (config 2: H 40, N 12, M 143; tau 0.1, lambda 2, g_ref 0.2)
+    wl = config(2)
+    inp = make_inputs(wl, "cuda")
+    layer = layer_for(wl)
+    p = layer.importance(inp.Q, inp.K)
+    H, N, M = wl.heads, wl.n_q_blocks, wl.n_kv_blocks
+    counts = torch.empty(H, N, 6, dtype=torch.int32, device="cuda")
+    prm = rbs.route_params(2.0, 0.1, 0.2, 0.9, 0.9, 80, 150)
+    t_a = _time_us(lambda: rbs.velox_route_audit(p, inp.g, H, N, M, prm, 50, 80, counts))
+    print(json.dumps({"variant": "audit", "config": "audit H40 N12 M143", "audit_us": t_a,
+                      **audit_metrics(counts, M), "random_expectation": 50 / M}), flush=True)
+    del inp, layer
+
+    # 2. model-only (lambda = 0) vs fused routing at chunk-48
+    wl = config(3)
+    inp = make_inputs(wl, "cuda")
+    out = {"variant": "model_only_vs_fused", "config": "chunk48 H40 N48 M2256"}
+    for name, lam in (("fused", wl.params.lam), ("model_only", 0.0)):
+        layer = layer_for(wl)
+        layer.prm = rbs.route_params(lam, wl.params.tau, wl.params.g_ref, wl.params.theta_cov,
+                                     wl.params.theta_unc, wl.params.k_cov, wl.params.k_unc)
+        layer.importance(inp.Q, inp.K)
+        t_r = _time_us(lambda: layer.route(inp.g, inp.covered), reps=20)
+        t_att = _time_us(lambda: layer.attend(inp.Q, inp.K, inp.V), reps=10)
+        out[name + "_route_us"] = t_r
+        out[name + "_attn_us"] = t_att
+        out[name + "_mean_route_len"] = float(layer.route_len.float().mean().item())
+        del layer
+    print(json.dumps(out), flush=True)
+    del inp
+
+    # 3. THW-linear vs Gilbert: neighbour table at the chunk-48 lattice
+    T, Hl, Wl, b, nc = 4, 32, 48, 128, 48
+    Nq = T * Hl * Wl // b
+    ids = torch.empty(Nq, 64, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(Nq, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = {"variant": "thw_linear_vs_gilbert", "lattice": "T4 32x48 b128, 48 chunks"}
+    for name, fn in (("gilbert", rbs.velox_gilbert_order), ("thw", rbs.velox_thw_linear_order)):
+        call = lambda: fn(T, Hl, Wl, nc, b, nc - 1, 0, (nc - 1) * Nq, nbr_ids=ids, nbr_cnt=cnt,
+                          S_max=64, dev_status=st)
+        out[name + "_nbr_us"] = _time_us(call)
+        # safeguards within the whole lattice (the cache holding every chunk)
+        fn(T, Hl, Wl, nc, b, nc - 2, 0, nc * Nq, nbr_ids=ids, nbr_cnt=cnt, S_max=64,
+           dev_status=st)
+        torch.cuda.synchronize()
+        out[name + "_mean_safeguards"] = float(cnt.float().mean().item())
+    out["dev_status"] = int(st.item())
+    print(json.dumps(out), flush=True)
+
+
 def run_layers(args):
     """Full denoising step at chunk 48: `args.layers` layers with independent
     per-layer inputs (seeded per layer), regenerated into reused buffers
@@ -608,6 +670,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="history-length sweep: routed vs dense attention per M (extra lines)")
+    ap.add_argument("--variants", action="store_true",
+                    help="audit, model-only routing and THW-linear comparisons")
     ap.add_argument("--geometry", action="store_true",
                     help="time slab overlap and coverage at the chunk-48 shape")
     ap.add_argument("--two-phase", action="store_true",
@@ -632,6 +696,9 @@ def main():
             return
         if args.geometry:
             run_geometry(args)
+            return
+        if args.variants:
+            run_variants(args)
             return
         if args.two_phase:
             run_two_phase(args)

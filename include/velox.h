@@ -485,13 +485,19 @@ VELOX_API velox_status velox_slab_table(const float *depth, const float *conf,
  * even count, fp64 rounded to fp32) of the first source, newest first, that
  * gives the token >= k_warp samples; 0 (a hole) if none does.  A camera index
  * out of range flags VELOX_DEV_BAD_CAMERA and that source (target) is
- * skipped (left 0).  Requires H W s^2 <= 32768.
+ * skipped (left 0).  ws: caller-owned device workspace of at least
+ * velox_multiwarp_workspace_size bytes (the per-source medians), else
+ * VELOX_ERR_WORKSPACE.  Requires H W s^2 <= 32768 and H W <= 8192.
  */
 VELOX_API velox_status velox_multiwarp(const velox_camera *cams, int n_cams,
                                        const float *src_depth, const int32_t *src_cam, int S,
                                        const int32_t *tgt_cam, int n_tgt, int H, int W, int s,
-                                       int k_warp, float *zq, int32_t *dev_status,
-                                       velox_stream_t stream);
+                                       int k_warp, float *zq, void *ws, size_t ws_bytes,
+                                       int32_t *dev_status, velox_stream_t stream);
+
+/* Bytes of workspace velox_multiwarp needs: 4 S n_tgt H W. */
+VELOX_API velox_status velox_multiwarp_workspace_size(int S, int n_tgt, int H, int W,
+                                                      size_t *bytes);
 
 #ifdef __cplusplus
 }

@@ -43,7 +43,7 @@ EXPORTS = ("velox_status_string", "velox_abi_version", "velox_gilbert_order",
            "velox_block_sparse_attn", "velox_block_importance_noalloc",
            "velox_route_schedule", "velox_two_phase_attn", "velox_slab_overlap",
            "velox_coverage", "velox_route_audit", "velox_thw_linear_order",
-           "velox_slab_table", "velox_multiwarp")
+           "velox_slab_table", "velox_multiwarp", "velox_multiwarp_workspace_size")
 
 
 class VeloxError(RuntimeError):
@@ -97,7 +97,10 @@ def _load() -> ctypes.CDLL:
     lib.velox_slab_table.argtypes = [P, P, P, I, I, I, I, I, P, I, I, I, I, F, I, D, D, P, P, P,
                                      P]
     lib.velox_multiwarp.restype = I
-    lib.velox_multiwarp.argtypes = [P, I, P, P, I, P, I, I, I, I, I, P, P, P]
+    lib.velox_multiwarp.argtypes = [P, I, P, P, I, P, I, I, I, I, I, P, P, ctypes.c_size_t, P,
+                                    P]
+    lib.velox_multiwarp_workspace_size.restype = I
+    lib.velox_multiwarp_workspace_size.argtypes = [I, I, I, I, ctypes.POINTER(ctypes.c_size_t)]
     lib.velox_two_phase_attn.restype = I
     lib.velox_two_phase_attn.argtypes = [P, P, P, P, P, P, I, P, P, I, I, I, I, I, I, F, P, P, P,
                                          P]
@@ -251,9 +254,16 @@ def velox_slab_table(depth, conf, mask, F, frame_base, H, W, s, cell_of_rank, n_
     _check("velox_slab_table", st)
 
 
+def velox_multiwarp_workspace_size(S, n_tgt, H, W) -> int:
+    out = ctypes.c_size_t(0)
+    _check("velox_multiwarp_workspace_size",
+           _lib.velox_multiwarp_workspace_size(S, n_tgt, H, W, ctypes.byref(out)))
+    return int(out.value)
+
+
 def velox_multiwarp(cams, n_cams, src_depth, src_cam, S, tgt_cam, n_tgt, H, W, s, k_warp, zq,
-                    dev_status, stream=None):
+                    ws, dev_status, stream=None):
     st = _lib.velox_multiwarp(_ptr(cams), n_cams, _ptr(src_depth), _ptr(src_cam), S,
-                              _ptr(tgt_cam), n_tgt, H, W, s, k_warp, _ptr(zq), _ptr(dev_status),
-                              _stream(stream))
+                              _ptr(tgt_cam), n_tgt, H, W, s, k_warp, _ptr(zq), _ptr(ws),
+                              ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream))
     _check("velox_multiwarp", st)

@@ -41,6 +41,8 @@ cudaError_t launch_coverage(const velox_camera *cams, int n_cams, const velox_sl
                             cudaStream_t stream);
 int audit_max_blocks();
 int multiwarp_max_samples();
+int multiwarp_max_tokens();
+size_t multiwarp_ws_bytes(int S, int n_tgt, int H, int W);
 int slab_table_max_samples();
 cudaError_t launch_slab_table(const float *depth, const float *conf, const uint8_t *mask, int F,
                               int frame_base, int H, int W, int s, const int32_t *cell_of_rank,
@@ -49,8 +51,8 @@ cudaError_t launch_slab_table(const float *depth, const float *conf, const uint8
                               float *token_uvz, int32_t *dev_status, cudaStream_t stream);
 cudaError_t launch_multiwarp(const velox_camera *cams, int n_cams, const float *src_depth,
                              const int32_t *src_cam, int S, const int32_t *tgt_cam, int n_tgt,
-                             int H, int W, int s, int k_warp, float *zq, int32_t *dev_status,
-                             cudaStream_t stream);
+                             int H, int W, int s, int k_warp, float *zq, void *ws,
+                             int32_t *dev_status, cudaStream_t stream);
 cudaError_t launch_audit(const float *p, const float *g, int H, int N, int M, double lam,
                          double tau, double g_ref, int k_geo, int k_fuse, int32_t *counts,
                          cudaStream_t stream);
@@ -382,20 +384,28 @@ velox_status velox_slab_table(const float *depth, const float *conf, const uint8
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
+velox_status velox_multiwarp_workspace_size(int S, int n_tgt, int H, int W, size_t *bytes) {
+  if (!bytes || S <= 0 || n_tgt <= 0 || H <= 0 || W <= 0) return VELOX_ERR_INVALID_ARG;
+  *bytes = velox::multiwarp_ws_bytes(S, n_tgt, H, W);
+  return VELOX_OK;
+}
+
 velox_status velox_multiwarp(const velox_camera *cams, int n_cams, const float *src_depth,
                              const int32_t *src_cam, int S, const int32_t *tgt_cam, int n_tgt,
-                             int H, int W, int s, int k_warp, float *zq, int32_t *dev_status,
-                             velox_stream_t stream) {
+                             int H, int W, int s, int k_warp, float *zq, void *ws,
+                             size_t ws_bytes, int32_t *dev_status, velox_stream_t stream) {
   if (!cams || !src_depth || !src_cam || !tgt_cam || !zq || !dev_status)
     return VELOX_ERR_INVALID_ARG;
   if (n_cams <= 0 || S <= 0 || n_tgt <= 0 || H <= 0 || W <= 0 || s <= 0 || k_warp < 1)
     return VELOX_ERR_INVALID_ARG;
-  if ((long long)H * W * s * s > velox::multiwarp_max_samples() || n_tgt > 65535)
+  if ((long long)H * W * s * s > velox::multiwarp_max_samples() ||
+      (long long)H * W > velox::multiwarp_max_tokens() || n_tgt > 65535 || S > 65535)
     return VELOX_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < velox::multiwarp_ws_bytes(S, n_tgt, H, W)) return VELOX_ERR_WORKSPACE;
   velox_status st = check_device();
   if (st != VELOX_OK) return st;
   return from_cuda(velox::launch_multiwarp(cams, n_cams, src_depth, src_cam, S, tgt_cam, n_tgt, H,
-                                           W, s, k_warp, zq, dev_status,
+                                           W, s, k_warp, zq, ws, dev_status,
                                            reinterpret_cast<cudaStream_t>(stream)));
 }
 

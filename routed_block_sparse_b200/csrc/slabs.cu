@@ -11,13 +11,14 @@
 //                       percentiles (linear interpolation between order
 //                       statistics, fp64) of its reliable samples, sorted in
 //                       shared memory by a bitonic network.
-//   multiwarp_kernel    one CTA per (target frame, tile of 256 target
-//                       tokens): the source frames are forward-warped newest
-//                       first; a token takes the median of the first source
-//                       that gives it at least k_warp samples.  Per source the
-//                       samples landing in the tile are counted, and only when
-//                       some open token qualifies are they warped again and
-//                       gathered by token (a counting sort) for the medians.
+//   multiwarp_scatter   one CTA per (source frame, target frame): every
+//                       source sample is forward-warped, the samples are
+//                       counted per target token, warped again and gathered by
+//                       token (a counting sort in shared memory), and each
+//                       token with at least k_warp samples gets their median
+//                       in the workspace (-1 otherwise).
+//   multiwarp_select    one thread per target token: the median of the
+//                       newest source that has one, else 0 (a hole).
 //
 // The warp of a sample uses explicitly rounded fp32 operations in the same
 // order as the coverage test, so the target token, an integer decided by
@@ -156,8 +157,6 @@ __global__ void __launch_bounds__(kThreads) slab_table_kernel(SlabArgs a) {
 
 // ---------------------------------------------------------------- multiwarp
 
-constexpr int kTile = 256;  // target tokens per CTA
-
 struct WarpArgs {
   const velox_camera *cams;
   int n_cams;
@@ -165,7 +164,9 @@ struct WarpArgs {
   const int32_t *src_cam;  // [S], newest first
   int S;
   const int32_t *tgt_cam;  // [n_tgt]
+  int n_tgt;
   int H, W, s, k_warp;
+  float *med;              // workspace [n_tgt][S][H W]: median or -1
   float *zq;               // [n_tgt][H][W]
   int32_t *dev_status;
 };
@@ -201,71 +202,68 @@ __device__ __forceinline__ int warp_one(const velox_camera &cs, const velox_came
   return (int)floorf(pv) * W + (int)floorf(pu);
 }
 
-__global__ void __launch_bounds__(kThreads) multiwarp_kernel(WarpArgs a) {
-  extern __shared__ float s_vals[];  // [H s W s]: one source's samples in the tile
-  __shared__ int s_cnt[kTile], s_off[kTile], s_fill[kTile];
-  __shared__ int s_wsum[kThreads / 32];
-  const int tgt = blockIdx.y;
-  const int HW = a.H * a.W;
-  const int tile0 = blockIdx.x * kTile;
-  const int tok = tile0 + threadIdx.x;  // kThreads == kTile: one token per thread
-  const int Hs = a.H * a.s, Ws = a.W * a.s, n_smp = Hs * Ws;
-  const int tc = a.tgt_cam[tgt];
-  const bool tgt_ok = tc >= 0 && tc < a.n_cams;
-  if (!tgt_ok && threadIdx.x == 0) flag_error(a.dev_status, VELOX_DEV_BAD_CAMERA);
-  bool open = tok < HW;  // still waiting for its depth
-  float zq = 0.f;
-  for (int k = 0; k < a.S && tgt_ok; ++k) {
-    if (!__syncthreads_or(open)) break;
-    const int sc = a.src_cam[k];
-    if (sc < 0 || sc >= a.n_cams) {
-      if (threadIdx.x == 0) flag_error(a.dev_status, VELOX_DEV_BAD_CAMERA);
-      continue;
-    }
-    const velox_camera cs = a.cams[sc], ct = a.cams[tc];
-    const float *src = a.src_depth + (size_t)k * n_smp;
-    s_cnt[threadIdx.x] = 0;
-    s_fill[threadIdx.x] = 0;
+// Dynamic shared memory: cnt[HW] int, off[HW] int, vals[H s W s] float.
+__global__ void __launch_bounds__(kThreads) multiwarp_scatter_kernel(WarpArgs a) {
+  extern __shared__ int s_mw[];
+  __shared__ int s_part[kThreads];
+  const int k = blockIdx.x, tgt = blockIdx.y;
+  const int HW = a.H * a.W, Ws = a.W * a.s, n_smp = a.H * a.s * Ws;
+  int *cnt = s_mw, *off = s_mw + HW;
+  float *vals = reinterpret_cast<float *>(s_mw + 2 * HW);
+  float *med = a.med + ((size_t)tgt * a.S + k) * HW;
+  const int sc = a.src_cam[k], tc = a.tgt_cam[tgt];
+  if (sc < 0 || sc >= a.n_cams || tc < 0 || tc >= a.n_cams) {
+    if (threadIdx.x == 0) flag_error(a.dev_status, VELOX_DEV_BAD_CAMERA);
+    for (int t = threadIdx.x; t < HW; t += kThreads) med[t] = -1.f;
+    return;
+  }
+  const velox_camera cs = a.cams[sc], ct = a.cams[tc];
+  const float *src = a.src_depth + (size_t)k * n_smp;
+  for (int t = threadIdx.x; t < HW; t += kThreads) cnt[t] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_smp; i += kThreads) {
+    const float z = src[i];
+    if (!(z > 0.f)) continue;
+    float dt;
+    const int t = warp_one(cs, ct, i % Ws, i / Ws, z, a.s, a.H, a.W, &dt);
+    if (t >= 0) atomicAdd(&cnt[t], 1);
+  }
+  __syncthreads();
+  // exclusive scan of cnt: thread p owns a contiguous run of tokens
+  const int run = (HW + kThreads - 1) / kThreads;
+  const int lo = min(HW, (int)threadIdx.x * run), hi = min(HW, lo + run);
+  int mine = 0;
+  for (int t = lo; t < hi; ++t) mine += cnt[t];
+  s_part[threadIdx.x] = mine;
+  __syncthreads();
+  for (int o = 1; o < kThreads; o <<= 1) {
+    const int v = threadIdx.x >= (unsigned)o ? s_part[threadIdx.x - o] : 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < n_smp; i += kThreads) {
-      const float z = src[i];
-      if (!(z > 0.f)) continue;
-      float dt;
-      const int t = warp_one(cs, ct, i % Ws, i / Ws, z, a.s, a.H, a.W, &dt);
-      if (t >= tile0 && t < tile0 + kTile) atomicAdd(&s_cnt[t - tile0], 1);
-    }
+    s_part[threadIdx.x] += v;
     __syncthreads();
-    const int cnt = s_cnt[threadIdx.x];
-    const bool take = open && cnt >= a.k_warp;
-    if (!__syncthreads_or(take)) continue;
-    // exclusive scan of the counts -> offsets
-    int incl = cnt;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    if (lane == 31) s_wsum[warp] = incl;
-    __syncthreads();
-    int before = 0;
-    for (int w = 0; w < warp; ++w) before += s_wsum[w];
-    s_off[threadIdx.x] = before + incl - cnt;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n_smp; i += kThreads) {
-      const float z = src[i];
-      if (!(z > 0.f)) continue;
-      float dt;
-      const int t = warp_one(cs, ct, i % Ws, i / Ws, z, a.s, a.H, a.W, &dt);
-      if (t >= tile0 && t < tile0 + kTile) {
-        const int lt = t - tile0;
-        s_vals[s_off[lt] + atomicAdd(&s_fill[lt], 1)] = dt;
-      }
-    }
-    __syncthreads();
-    if (take) {
-      float *v = s_vals + s_off[threadIdx.x];
-      for (int x = 1; x < cnt; ++x) {  // insertion sort of this token's samples
+  }
+  int acc = s_part[threadIdx.x] - mine;
+  for (int t = lo; t < hi; ++t) {
+    off[t] = acc;
+    acc += cnt[t];
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < HW; t += kThreads) cnt[t] = 0;  // reused as fill counters
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_smp; i += kThreads) {
+    const float z = src[i];
+    if (!(z > 0.f)) continue;
+    float dt;
+    const int t = warp_one(cs, ct, i % Ws, i / Ws, z, a.s, a.H, a.W, &dt);
+    if (t >= 0) vals[off[t] + atomicAdd(&cnt[t], 1)] = dt;
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < HW; t += kThreads) {
+    const int n = cnt[t];
+    float m = -1.f;
+    if (n >= a.k_warp) {
+      float *v = vals + off[t];
+      for (int x = 1; x < n; ++x) {  // insertion sort of this token's samples
         const float key = v[x];
         int y = x - 1;
         while (y >= 0 && v[y] > key) {
@@ -274,16 +272,28 @@ __global__ void __launch_bounds__(kThreads) multiwarp_kernel(WarpArgs a) {
         }
         v[y + 1] = key;
       }
-      if (cnt & 1) {
-        zq = v[cnt / 2];
-      } else {
-        zq = __double2float_rn(__dmul_rn(__dadd_rn((double)v[cnt / 2 - 1], (double)v[cnt / 2]), 0.5));
-      }
-      open = false;
+      m = (n & 1) ? v[n / 2]
+                  : __double2float_rn(
+                        __dmul_rn(__dadd_rn((double)v[n / 2 - 1], (double)v[n / 2]), 0.5));
     }
-    __syncthreads();
+    med[t] = m;
   }
-  if (tok < HW) a.zq[(size_t)tgt * HW + tok] = zq;
+}
+
+__global__ void multiwarp_select_kernel(WarpArgs a) {
+  const int HW = a.H * a.W;
+  const int tgt = blockIdx.y;
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= HW) return;
+  float z = 0.f;
+  for (int k = 0; k < a.S; ++k) {  // newest source first
+    const float m = a.med[((size_t)tgt * a.S + k) * HW + t];
+    if (m >= 0.f) {
+      z = m;
+      break;
+    }
+  }
+  a.zq[(size_t)tgt * HW + t] = z;
 }
 
 }  // namespace
@@ -326,10 +336,14 @@ cudaError_t launch_slab_table(const float *depth, const float *conf, const uint8
   return cudaGetLastError();
 }
 
+size_t multiwarp_ws_bytes(int S, int n_tgt, int H, int W) {
+  return sizeof(float) * (size_t)S * n_tgt * H * W;
+}
+
 cudaError_t launch_multiwarp(const velox_camera *cams, int n_cams, const float *src_depth,
                              const int32_t *src_cam, int S, const int32_t *tgt_cam, int n_tgt,
-                             int H, int W, int s, int k_warp, float *zq, int32_t *dev_status,
-                             cudaStream_t stream) {
+                             int H, int W, int s, int k_warp, float *zq, void *ws,
+                             int32_t *dev_status, cudaStream_t stream) {
   WarpArgs a;
   a.cams = cams;
   a.n_cams = n_cams;
@@ -337,24 +351,29 @@ cudaError_t launch_multiwarp(const velox_camera *cams, int n_cams, const float *
   a.src_cam = src_cam;
   a.S = S;
   a.tgt_cam = tgt_cam;
+  a.n_tgt = n_tgt;
   a.H = H;
   a.W = W;
   a.s = s;
   a.k_warp = k_warp;
+  a.med = static_cast<float *>(ws);
   a.zq = zq;
   a.dev_status = dev_status;
-  const size_t smem = sizeof(float) * (size_t)H * W * s * s;
+  const size_t smem = sizeof(int) * 2 * (size_t)H * W + sizeof(float) * (size_t)H * W * s * s;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(multiwarp_kernel,
+    cudaError_t e = cudaFuncSetAttribute(multiwarp_scatter_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  dim3 grid((H * W + kTile - 1) / kTile, n_tgt);
-  multiwarp_kernel<<<grid, kThreads, smem, stream>>>(a);
+  multiwarp_scatter_kernel<<<dim3(S, n_tgt), kThreads, smem, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  multiwarp_select_kernel<<<dim3((H * W + 255) / 256, n_tgt), 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
 int multiwarp_max_samples() { return 32768; }
+int multiwarp_max_tokens() { return 8192; }
 int slab_table_max_samples() { return 16384; }
 
 }  // namespace velox

@@ -111,3 +111,18 @@ def layer_for(wl, device="cuda", **kw) -> RoutedLayer:
                        prev_begin=wl.prev_begin, prev_count=wl.prev_count,
                        lattice=wl.lattice, q_chunk=wl.q_chunk,
                        cache_first_block=wl.cache_first_block, device=device, **kw)
+
+
+def audit_metrics(counts: torch.Tensor, M: int, k_geo: int = 50, k_fuse: int = 80) -> dict:
+    """Pooled ratios (sums over all rows) from the six per-row counts that
+    velox_route_audit writes: R_geo, R_50, top-k_fuse recall of the
+    positive-overlap blocks for the model's p and for the fused weight, and
+    the fraction of the fused top-k_fuse not in the model's."""
+    c = counts.reshape(-1, 6).to(torch.int64)
+    rows = c.shape[0]
+    t = c.sum(dim=0).tolist()
+    n_pos = t[0]
+    ratio = (lambda x: x / n_pos) if n_pos else (lambda x: float("nan"))
+    return {"R_geo": ratio(t[1]), "R_50": t[2] / (rows * min(k_geo, M)),
+            "recall_top_fuse_model": ratio(t[3]), "recall_top_fuse_fused": ratio(t[4]),
+            "changed_fraction": t[5] / (rows * min(k_fuse, M)), "positive_blocks": n_pos}

@@ -92,11 +92,13 @@ def test_slab_table_flags_blocks_outside_the_frames(lib):
 def _gpu_multiwarp(cams, src_depth, src_cam, tgt_cam, H, W, s, k_warp):
     zq = torch.full((len(tgt_cam), H, W), -1.0, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(rbs.velox_multiwarp_workspace_size(len(src_cam), len(tgt_cam), H, W),
+                     dtype=torch.uint8, device="cuda")
     rbs.velox_multiwarp(torch.from_numpy(cams).cuda(), cams.shape[0],
                         torch.from_numpy(np.ascontiguousarray(src_depth)).cuda(),
                         torch.tensor(src_cam, dtype=torch.int32, device="cuda"), len(src_cam),
                         torch.tensor(tgt_cam, dtype=torch.int32, device="cuda"), len(tgt_cam),
-                        H, W, s, k_warp, zq, st)
+                        H, W, s, k_warp, zq, ws, st)
     torch.cuda.synchronize()
     return zq.cpu().numpy(), int(st.item())
 
@@ -127,7 +129,7 @@ def test_multiwarp_chunk48_frame(lib):
 def test_multiwarp_bad_camera_is_flagged(lib):
     H, W, s = 4, 8, 2
     r = make_rollout(1, 4, H, W, s)
-    zq, st = _gpu_multiwarp(r.cams, r.depth[[2, 1]], [2, 99], [3], H, W, s, 2)
+    zq, st = _gpu_multiwarp(r.cams, r.depth[[1, 2]], [99, 2], [3], H, W, s, 2)
     assert st & rbs.DEV_BAD_CAMERA
     ref = osl.multiwarp(r.cams, r.depth[[2]], [2], 3, H, W, s, 2)
     assert np.array_equal(zq[0], ref)
