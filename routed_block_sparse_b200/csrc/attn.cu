@@ -19,15 +19,21 @@
 //               PV_{j-1} has completed it issues S_{j+2} = Q K_{j+2}^T into the
 //               buffer P_{j-1} occupied, then O += P_j V_j (A = P from TMEM,
 //               B = V from shared memory) once the softmax of tile j is done.
-//   warps 2-5   softmax: one query row per thread (its TMEM lane).  One
-//               TMEM read of the S row, row max with three-input max, scaled
-//               exponent arguments and the row sum in packed fp32x2
-//               arithmetic, exponentials on MUFU, P_j packed to bf16 into the
-//               first 64 columns of its own S buffer.  The running max is
-//               only moved (and O rescaled in TMEM, after waiting for
-//               PV_{j-1}) when it grows by more than 2^8; otherwise the stale
-//               max is kept, which is exact because O and the row sum always
-//               use the same max.  Epilogue: O / l -> bf16, lse.
+//   warps 2-9   softmax: two threads per query row (the row's TMEM lane, in
+//               warps w and w + 4), each owning 64 of the tile's 128
+//               columns, so every scheduler has two softmax warps to switch
+//               between.  One TMEM read of the half row, a three-input max,
+//               the two half maxima exchanged through shared memory (an
+//               mbarrier per S buffer), scaled exponent arguments and the
+//               row sum in packed fp32x2 arithmetic, exponentials on MUFU,
+//               P_j packed to bf16 into the first 64 columns of its own S
+//               buffer (half h writes columns 32h..32h+31, after both halves
+//               have read their S).  The running max is only moved (and O
+//               rescaled in TMEM, each half its 64 channels, after waiting
+//               for PV_{j-1}) when it grows by more than 2^8; otherwise the
+//               stale max is kept, which is exact because O and the row sum
+//               always use the same max.  Each half keeps its own partial row
+//               sum; the epilogue adds them: O / l -> bf16, lse.
 // A pre-pass compacts the route into shared memory, skipping ids outside
 // [0, M) and repeats (flagged in dev_status).
 //
@@ -47,7 +53,8 @@ namespace {
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // tokens per KV tile
 constexpr int D = 128;   // head dim
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // TMA warp, MMA warp, 8 softmax warps
+constexpr int kSoftThreads = 256;
 constexpr uint32_t kTileBytes = BN * D * 2;      // 32 KB
 constexpr uint32_t kHalfBytes = kTileBytes / 2;  // one 64-channel box
 constexpr int kMaxRoute = VELOX_MAX_ROUTE;
@@ -61,8 +68,10 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest tolerated grow
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffRing = kOffQ + kTileBytes;
 // barriers, misc and the dynamic tail follow the ring (offset set at launch)
-constexpr uint32_t kNumBars = 1 + 2 * kMaxSlots + 3 * kSBufs + 1;
+constexpr uint32_t kNumBars = 1 + 2 * kMaxSlots + 3 * kSBufs + 1 + kSBufs + 1;
 constexpr uint32_t kMiscBytes = 64;
+// half-row maxima, rounded up to bf16, in two alternating slots: [2][2][128]
+constexpr uint32_t kXchBytes = 2 * 2 * BM * 2;
 constexpr uint32_t kSmemLimit = 227 * 1024;
 
 struct AttnArgs {
@@ -79,6 +88,7 @@ struct AttnArgs {
   int32_t *dev_status;
   int nslot;              // K/V ring slots in use (4..kMaxSlots)
   uint32_t bar_offset;    // byte offset of the barriers from the aligned base
+  uint32_t xch_offset;    // half-row maxima exchange area (bf16 bits)
   uint32_t list_offset;   // route list (uint16)
   uint32_t bits_offset;   // id bitmap (uint32)
 };
@@ -105,6 +115,14 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// bf16 bits of finite x rounded towards +inf.
+__device__ __forceinline__ uint16_t bf16_round_up(float x) {
+  const uint32_t u = __float_as_uint(x);
+  uint32_t hi = u >> 16;
+  if ((u & 0xffffu) != 0u && (u >> 31) == 0u) hi += 1u;  // positive: away from 0; negative: toward 0
+  return static_cast<uint16_t>(hi);
+}
+
 // Warp-uniform bounded wait (tcgen05.ld/st after it are warp-collective).
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
@@ -127,7 +145,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *p_full = s_full + kSBufs;
   uint64_t *pv_done = p_full + kSBufs;
   uint64_t *mma_done = pv_done + kSBufs;
+  uint64_t *x_max = mma_done + 1;   // both half-row maxima of S buffer b written
+  uint64_t *x_fin = x_max + kSBufs;  // both partial row sums written
   uint8_t *misc = base + a.bar_offset + kNumBars * 8;
+  uint16_t *xch = reinterpret_cast<uint16_t *>(base + a.xch_offset);
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(misc);
   int *s_nvalid = reinterpret_cast<int *>(misc + 4);
   volatile int *s_abort = reinterpret_cast<volatile int *>(misc + 8);
@@ -154,10 +175,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < kSBufs; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 128);
+      mbar_init(&p_full[b], kSoftThreads);
       mbar_init(&pv_done[b], 1);
+      mbar_init(&x_max[b], kSoftThreads);
     }
     mbar_init(mma_done, 1);
+    mbar_init(x_fin, kSoftThreads);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -300,32 +323,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(mma_done, 0, &never);
     }
   } else {
-    // ================= softmax / epilogue (warps 2..5) =================
+    // ================= softmax / epilogue (warps 2..9) =================
     const int quarter = warp & 3;
+    const int hf = (warp - 2) >> 2;     // which 64 columns of the row
     const int r = quarter * 32 + lane;  // query row within the tile = TMEM lane
     const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float c = a.scale_log2;
-    float m_run = -INFINITY, l = 0.f;
+    float m_run = -INFINITY, l = 0.f;  // l: this half's partial row sum
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int b = j % kSBufs;
+      const uint32_t ph = (j / kSBufs) & 1;
       const uint32_t sb = trow + b * BN;
-      if (!warp_wait(&s_full[b], (j / kSBufs) & 1, s_abort)) { ok = false; break; }
+      if (!warp_wait(&s_full[b], ph, s_abort)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sv[128];
-      tmem_ld32(sb, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(sb + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      tmem_ld32(sb + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-      tmem_ld32(sb + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+      uint32_t sv[64];
+      tmem_ld32(sb + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(sb + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       tmem_wait_ld();
-      float mx[8];
+      float mx[4];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
+      for (int q = 0; q < 4; ++q) mx[q] = -INFINITY;
 #pragma unroll
-      for (int k = 0; k < 64; ++k)
-        mx[k & 7] = fmax3(mx[k & 7], __uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1]));
-      const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
-                             fmaxf(mx[6], mx[7]));
+      for (int k = 0; k < 32; ++k)
+        mx[k & 3] = fmax3(mx[k & 3], __uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1]));
+      // exchange the half maxima, each rounded up to bf16 so that both halves
+      // take the same (slightly larger, hence still exact) max; slot j & 1 is
+      // free again because the partner read it before arriving for tile j - 1.
+      // After this wait both halves have read their S columns, so P may
+      // overwrite columns 0..63 of the buffer.
+      const uint16_t mh = bf16_round_up(fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]));
+      xch[((j & 1) * 2 + hf) * BM + r] = mh;
+      tc_fence_before();
+      mbar_arrive(&x_max[b]);
+      if (!warp_wait(&x_max[b], ph, s_abort)) { ok = false; break; }
+      tc_fence_after();
+      const uint16_t mo = xch[((j & 1) * 2 + (hf ^ 1)) * BM + r];
+      const float mt = fmaxf(__uint_as_float(static_cast<uint32_t>(mh) << 16),
+                             __uint_as_float(static_cast<uint32_t>(mo) << 16));
       const float m_cand = fmaxf(m_run, mt * c);
       const bool grow = m_cand > m_run + kRescaleThreshold;  // always on the first tile
       const float m_use = grow ? m_cand : m_run;
@@ -336,61 +371,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!warp_wait(&pv_done[jp % kSBufs], (jp / kSBufs) & 1, s_abort)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t ov[32];
-          tmem_ld32(trow + kColO + cc * 32, ov);
+          const uint32_t oa = trow + kColO + hf * 64 + cc * 32;
+          tmem_ld32(oa, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
-          tmem_st32(trow + kColO + cc * 32, ov);
+          tmem_st32(oa, ov);
         }
       }
       // exponentials (arguments and row sum in packed pairs); P_j into the
       // first 64 columns of its S buffer: column t/2 holds elements t, t+1
       uint64_t sum2[2] = {0ull, 0ull};
       const uint64_t c2 = f2pack(c, c), nm2 = f2pack(-m_use, -m_use);
+      uint32_t pk[32];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const uint64_t x2 = ffma2(f2pack(__uint_as_float(sv[half * 64 + 2 * k]),
-                                           __uint_as_float(sv[half * 64 + 2 * k + 1])),
-                                    c2, nm2);
-          float x0, x1;
-          f2unpack(x2, x0, x1);
-          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-          sum2[k & 1] = fadd2(sum2[k & 1], f2pack(p0, p1));
-          pk[k] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(sb + half * 32, pk);
+      for (int k = 0; k < 32; ++k) {
+        const uint64_t x2 = ffma2(f2pack(__uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1])),
+                                  c2, nm2);
+        float x0, x1;
+        f2unpack(x2, x0, x1);
+        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+        sum2[k & 1] = fadd2(sum2[k & 1], f2pack(p0, p1));
+        pk[k] = pack_bf16x2(p0, p1);
       }
-      float sa, sb2, sc, sd;
+      tmem_st32(sb + hf * 32, pk);
+      float sa, sb2;
       f2unpack(fadd2(sum2[0], sum2[1]), sa, sb2);
       tmem_wait_st();
       l = l * alpha + (sa + sb2);
       m_run = m_use;
-      (void)sc;
-      (void)sd;
       tc_fence_before();
       mbar_arrive(&p_full[b]);
     }
-    // epilogue
-    uint16_t *orow = a.O + ((size_t)row * BM + r) * D;
+    // epilogue: the row sum is the sum of the two halves' partial sums
+    uint16_t *orow = a.O + ((size_t)row * BM + r) * D + hf * 64;
     bool have = ok && n > 0;
     if (have) {
       const int jl = n - 1;
       have = mbar_wait(&pv_done[jl % kSBufs], (jl / kSBufs) & 1, s_abort);
     }
+    // the Q tile is dead once the last PV is done: it carries the partial sums
+    float *lx = reinterpret_cast<float *>(sQ);
+    lx[hf * BM + r] = l;
+    mbar_arrive(x_fin);
+    const bool fin = mbar_wait(x_fin, 0, s_abort);
+    const float l_row = l + lx[(hf ^ 1) * BM + r];
     // tcgen05.ld is warp-collective: decide once for the whole warp
-    const bool good = __all_sync(0xffffffffu, have && !*s_abort);
+    const bool good = __all_sync(0xffffffffu, have && fin && !*s_abort);
     tc_fence_after();
-    const float inv = good ? 1.0f / l : 0.f;
+    const float inv = good ? 1.0f / l_row : 0.f;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
+    for (int cc = 0; cc < 2; ++cc) {
       uint32_t ov[32];
       if (good) {
-        tmem_ld32(trow + kColO + cc * 32, ov);
+        tmem_ld32(trow + kColO + hf * 64 + cc * 32, ov);
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -406,7 +442,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint4 *>(orow + cc * 32 + q * 8) = v;
       }
     }
-    if (a.lse) a.lse[(size_t)row * BM + r] = good ? (m_run + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    if (a.lse && hf == 0)
+      a.lse[(size_t)row * BM + r] = good ? (m_run + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
   }
 
   if (*s_abort && threadIdx.x == 0) flag_error(a.dev_status, VELOX_DEV_WAIT_TIMEOUT);
@@ -483,12 +520,17 @@ cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
   // tail after the ring: barriers, misc, route list (uint16), id bitmap
   const uint32_t list_bytes = route_ids ? ((uint32_t)R_max * 2u + 15u) & ~15u : 0u;
   const uint32_t bits_bytes = route_ids ? (uint32_t)((M + 31) / 32) * 4u : 0u;
-  const uint32_t tail = kNumBars * 8 + kMiscBytes + list_bytes + bits_bytes;
+  const uint32_t tail = kNumBars * 8 + kMiscBytes + kXchBytes + list_bytes + bits_bytes;
   int nslot = kMaxSlots;
   while (nslot > 4 && kOffRing + nslot * kTileBytes + tail + 1024 > kSmemLimit) --nslot;
+  // loads go K_0, V_0, K_1, V_1, ... round the ring; load li reuses the slot
+  // of load li - nslot.  With an odd count K_{j+3} would reuse V_j's slot and
+  // could not start before PV_j, just when S_{j+3} is wanted: keep it even.
+  nslot &= ~1;
   a.nslot = nslot;
   a.bar_offset = kOffRing + nslot * kTileBytes;
-  a.list_offset = a.bar_offset + kNumBars * 8 + kMiscBytes;
+  a.xch_offset = a.bar_offset + kNumBars * 8 + kMiscBytes;
+  a.list_offset = a.xch_offset + kXchBytes;
   a.bits_offset = a.list_offset + list_bytes;
   const size_t smem = (size_t)a.bits_offset + bits_bytes + 1024;  // + alignment slack
   if (smem > kSmemLimit) return cudaErrorInvalidConfiguration;
