@@ -7,21 +7,26 @@
 // attention restricted to the tokens of the listed tiles, computed with the
 // FlashAttention online-softmax recurrence over tiles.
 //
-// sm_100a design: one CTA per (head, query block), one CTA per SM, all 512
-// TMEM columns: three S buffers (128 columns each) and the O accumulator.
+// sm_100a design: one CTA per (head, query block), one CTA per SM; TMEM holds
+// two S buffers (128 columns each), the query tile Q (64 columns of bf16
+// pairs, the A operand of S = Q K^T) and the O accumulator, so the score
+// product reads only K from shared memory.
 // CTAs take rows in the order `row_order` gives (longest routes first, from
 // velox_route_schedule), so the last wave is made of short rows.
-//   warp 0      TMA producer: Q once, then K_0, V_0, K_1, V_1, ... of the
-//               route into a ring of 32 KB slots (128-byte swizzle, two
-//               64-channel boxes per tile).
-//   warp 1      TMEM allocator and the single tcgen05.mma issuer.  It keeps
-//               the score products two tiles ahead of the softmax: as soon as
-//               PV_{j-1} has completed it issues S_{j+2} = Q K_{j+2}^T into the
-//               buffer P_{j-1} occupied, then O += P_j V_j (A = P from TMEM,
-//               B = V from shared memory) once the softmax of tile j is done.
+//   warp 0      TMA producer: K_0, V_0, K_1, V_1, ... of the route into a
+//               ring of 32 KB slots (128-byte swizzle, two 64-channel boxes
+//               per tile).
+//   warp 1      TMEM allocator and the single tcgen05.mma issuer.  S_j =
+//               Q K_j^T (A = Q from TMEM, B = K from shared memory) goes into
+//               buffer j mod 2; once the softmax of tile j is done it issues
+//               O += P_j V_j (A = P from TMEM, B = V from shared memory) and,
+//               as soon as that has completed, S_{j+2} into the same buffer,
+//               so the score product of tile j+1 runs under the softmax of
+//               tile j.
 //   warps 2-9   softmax: two threads per query row (the row's TMEM lane, in
 //               warps w and w + 4), each owning 64 of the tile's 128
-//               columns, so every scheduler has two softmax warps to switch
+//               columns; at the start each writes its half of the row's Q
+//               into TMEM, so every scheduler has two softmax warps to switch
 //               between.  One TMEM read of the half row, a three-input max,
 //               the two half maxima exchanged through shared memory (an
 //               mbarrier per S buffer), scaled exponent arguments and the
@@ -59,22 +64,24 @@ constexpr uint32_t kTileBytes = BN * D * 2;      // 32 KB
 constexpr uint32_t kHalfBytes = kTileBytes / 2;  // one 64-channel box
 constexpr int kMaxRoute = VELOX_MAX_ROUTE;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kSBufs = 3;         // S/P buffers in TMEM, columns 0, 128, 256
+constexpr int kSBufs = 2;         // S/P buffers in TMEM, columns 0 and 128
+constexpr uint32_t kColQ = 256;   // Q (bf16 pairs, 64 columns)
 constexpr uint32_t kColO = 384;   // O accumulator (fp32, 128 columns)
 constexpr int kMaxSlots = 6;      // K/V ring slots of 32 KB
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest tolerated growth
 
 // shared-memory layout (offsets from a 1024-byte aligned base)
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffRing = kOffQ + kTileBytes;
+constexpr uint32_t kOffRing = 0;
 // barriers, misc and the dynamic tail follow the ring (offset set at launch)
 constexpr uint32_t kNumBars = 1 + 2 * kMaxSlots + 3 * kSBufs + 1 + kSBufs + 1;
 constexpr uint32_t kMiscBytes = 64;
-// half-row maxima, rounded up to bf16, in two alternating slots: [2][2][128]
-constexpr uint32_t kXchBytes = 2 * 2 * BM * 2;
+// half-row maxima, rounded up to bf16, in two alternating slots ([2][2][128]
+// bf16), then the two partial row sums of the epilogue ([2][128] fp32)
+constexpr uint32_t kXchBytes = 2 * 2 * BM * 2 + 2 * BM * 4;
 constexpr uint32_t kSmemLimit = 227 * 1024;
 
 struct AttnArgs {
+  const uint16_t *Q;         // [H][N * 128][128] bf16
   const int32_t *route_ids;  // null: dense
   const int32_t *route_len;
   const int32_t *row_order;  // null: row = blockIdx.x
@@ -129,13 +136,12 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+    attn_kernel(const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
                 const __grid_constant__ CUtensorMap tmVc, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-  uint8_t *sQ = base + kOffQ;
   uint8_t *ring = base + kOffRing;
   uint64_t *bar = reinterpret_cast<uint64_t *>(base + a.bar_offset);
   uint64_t *q_full = bar;
@@ -168,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- set-up: barriers, TMEM, route compaction
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    mbar_init(q_full, kSoftThreads);  // Q written to TMEM by the softmax threads
     for (int s = 0; s < kMaxSlots; ++s) {
       mbar_init(&slot_full[s], 1);
       mbar_init(&slot_empty[s], 1);
@@ -237,16 +243,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ================= TMA producer =================
     if (lane == 0 && n > 0) {
-      prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       if (a.n_cur > 0) {
         prefetch_tmap(&tmKc);
         prefetch_tmap(&tmVc);
       }
-      mbar_arrive_expect_tx(q_full, kTileBytes);
-      tma_load_3d(sQ, &tmQ, q_full, 0, i * BM, h);
-      tma_load_3d(sQ + kHalfBytes, &tmQ, q_full, 64, i * BM, h);
       int issued = 0;
       for (int li = 0; li < 2 * n; ++li) {  // load li: K_{li/2} (even) or V_{li/2} (odd)
         const int s = li % nslot;
@@ -266,7 +268,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // let the copies already in flight land before the CTA goes away
         // (each wait is bounded by the same time limit)
         volatile int never = 0;
-        mbar_wait(q_full, 0, &never);
         for (int li = issued - nslot < 0 ? 0 : issued - nslot; li < issued; ++li) {
           never = 0;
           mbar_wait(&slot_full[li % nslot], (li / nslot) & 1, &never);
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && n > 0) {
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false);
       constexpr uint32_t idPV = idesc_bf16_f32(BM, D, true);
-      const uint32_t qa = smem_u32(sQ), ra = smem_u32(ring);
+      const uint32_t ra = smem_u32(ring);
       auto issue_s = [&](int j) -> bool {
         const int li = 2 * j, s = li % nslot;
         if (!mbar_wait(&slot_full[s], (li / nslot) & 1, s_abort)) return false;
@@ -287,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sb = tmem + (j % kSBufs) * BN;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_bf16_ss(sb, kmajor_desc(qa, k), kmajor_desc(ka, k), idS, k > 0);
+          mma_bf16_ts(sb, tmem + kColQ + k * 8, kmajor_desc(ka, k), idS, k > 0);
         tc_commit(&s_full[j % kSBufs]);
         tc_commit(&slot_empty[s]);
         return true;
@@ -297,14 +298,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && n > 1) ok = issue_s(1);
       for (int j = 0; ok && j < n; ++j) {
         const int b = j % kSBufs;
-        if (j + 2 < n) {
-          // S_{j+2} goes into the buffer P_{j-1} occupied: PV_{j-1} must be done
-          if (j >= 1) {
-            const int jp = j - 1;
-            if (!mbar_wait(&pv_done[jp % kSBufs], (jp / kSBufs) & 1, s_abort)) break;
-          }
-          if (!issue_s(j + 2)) break;
-        }
         if (!mbar_wait(&p_full[b], (j / kSBufs) & 1, s_abort)) break;
         const int li = 2 * j + 1, s = li % nslot;
         if (!mbar_wait(&slot_full[s], (li / nslot) & 1, s_abort)) break;
@@ -316,6 +309,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16_ts(tmem + kColO, pb + k * 8, vmn_desc(va, k), idPV, (j > 0 || k > 0));
         tc_commit(&pv_done[b]);
         tc_commit(&slot_empty[s]);
+        if (j + 2 < n) {
+          // S_{j+2} goes into the buffer P_j occupies: PV_j must be done
+          if (!mbar_wait(&pv_done[b], (j / kSBufs) & 1, s_abort)) break;
+          if (!issue_s(j + 2)) break;
+        }
       }
       // all issued MMAs must be complete before TMEM is released
       tc_commit(mma_done);
@@ -331,6 +329,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = a.scale_log2;
     float m_run = -INFINITY, l = 0.f;  // l: this half's partial row sum
     bool ok = true;
+    if (n > 0) {
+      // this thread's half of Q row r into TMEM: bf16 pairs, element 2c in the
+      // low half of column c, as the A operand of S = Q K^T expects
+      const uint4 *qsrc = reinterpret_cast<const uint4 *>(
+          a.Q + (((size_t)h * a.N + i) * BM + r) * D + hf * 64);
+      uint32_t qv[32];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint4 v = __ldg(qsrc + q);
+        qv[4 * q + 0] = v.x;
+        qv[4 * q + 1] = v.y;
+        qv[4 * q + 2] = v.z;
+        qv[4 * q + 3] = v.w;
+      }
+      tmem_st32(trow + kColQ + hf * 32, qv);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    mbar_arrive(q_full);
     for (int j = 0; j < n; ++j) {
       const int b = j % kSBufs;
       const uint32_t ph = (j / kSBufs) & 1;
@@ -412,8 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int jl = n - 1;
       have = mbar_wait(&pv_done[jl % kSBufs], (jl / kSBufs) & 1, s_abort);
     }
-    // the Q tile is dead once the last PV is done: it carries the partial sums
-    float *lx = reinterpret_cast<float *>(sQ);
+    float *lx = reinterpret_cast<float *>(base + a.xch_offset + 2 * 2 * BM * 2);
     lx[hf * BM + r] = l;
     mbar_arrive(x_fin);
     const bool fin = mbar_wait(x_fin, 0, s_abort);
@@ -495,9 +511,9 @@ cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                         float softmax_scale, uint16_t *O, float *lse, int32_t *dev_status,
                         cudaStream_t stream, bool *map_failed) {
   *map_failed = false;
-  CUtensorMap mq, mk, mv, mkc, mvc;
+  CUtensorMap mk, mv, mkc, mvc;
   const bool cur = K_cur != nullptr && N_cur > 0;
-  if (!make_map(&mq, Q, N * BM, H) || !make_map(&mk, K, M * BN, H) ||
+  if (!make_map(&mk, K, M * BN, H) ||
       !make_map(&mv, V, M * BN, H) ||
       !make_map(&mkc, cur ? K_cur : K, cur ? N_cur * BN : M * BN, H) ||
       !make_map(&mvc, cur ? V_cur : V, cur ? N_cur * BN : M * BN, H)) {
@@ -505,6 +521,7 @@ cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
     return cudaErrorInvalidValue;
   }
   AttnArgs a;
+  a.Q = Q;
   a.route_ids = route_ids;
   a.route_len = route_len;
   a.row_order = row_order;
@@ -537,7 +554,7 @@ cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
   cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  attn_kernel<<<H * N, kThreads, smem, stream>>>(mq, mk, mv, mkc, mvc, a);
+  attn_kernel<<<H * N, kThreads, smem, stream>>>(mk, mv, mkc, mvc, a);
   return cudaGetLastError();
 }
 
