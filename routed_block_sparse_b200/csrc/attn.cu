@@ -7,38 +7,35 @@
 // attention restricted to the tokens of the listed tiles, computed with the
 // FlashAttention online-softmax recurrence over tiles.
 //
-// sm_100a design: one CTA per (head, query block), one CTA per SM; TMEM holds
-// two S buffers (128 columns each), the query tile Q (64 columns of bf16
-// pairs, the A operand of S = Q K^T) and the O accumulator, so the score
-// product reads only K from shared memory.
+// sm_100a design: one CTA per (head, query block), one CTA per SM.  The
+// tiles of the route are split into two interleaved chains, even and odd,
+// each with its own S buffer and its own O accumulator in TMEM (4 x 128
+// columns) and its own softmax warpgroup with its own running max and row
+// sum, so two tiles are in their softmax at once; the epilogue merges the
+// two partial results (FlashAttention's split-KV merge, inside the CTA).
 // CTAs take rows in the order `row_order` gives (longest routes first, from
 // velox_route_schedule), so the last wave is made of short rows.
-//   warp 0      TMA producer: K_0, V_0, K_1, V_1, ... of the route into a
-//               ring of 32 KB slots (128-byte swizzle, two 64-channel boxes
-//               per tile).
+//   warp 0      TMA producer: Q once, then K_0, V_0, K_1, V_1, ... of the
+//               route into a ring of 32 KB slots (128-byte swizzle, two
+//               64-channel boxes per tile).
 //   warp 1      TMEM allocator and the single tcgen05.mma issuer.  S_j =
-//               Q K_j^T (A = Q from TMEM, B = K from shared memory) goes into
-//               buffer j mod 2; once the softmax of tile j is done it issues
-//               O += P_j V_j (A = P from TMEM, B = V from shared memory) and,
-//               as soon as that has completed, S_{j+2} into the same buffer,
-//               so the score product of tile j+1 runs under the softmax of
-//               tile j.
-//   warps 2-9   softmax: two threads per query row (the row's TMEM lane, in
-//               warps w and w + 4), each owning 64 of the tile's 128
-//               columns; at the start each writes its half of the row's Q
-//               into TMEM, so every scheduler has two softmax warps to switch
-//               between.  One TMEM read of the half row, a three-input max,
-//               the two half maxima exchanged through shared memory (an
-//               mbarrier per S buffer), scaled exponent arguments and the
+//               Q K_j^T (both operands from shared memory) goes into buffer
+//               j mod 2; once the softmax of tile j is done it issues
+//               O_{j mod 2} += P_j V_j (A = P from TMEM, B = V from shared
+//               memory) and, as soon as that has completed, S_{j+2} into the
+//               same buffer.
+//   warps 2-5   softmax of the even tiles, warps 6-9 of the odd tiles: one
+//               query row per thread (its TMEM lane).  One TMEM read of the S
+//               row, a three-input max, scaled exponent arguments and the
 //               row sum in packed fp32x2 arithmetic, exponentials on MUFU,
 //               P_j packed to bf16 into the first 64 columns of its own S
-//               buffer (half h writes columns 32h..32h+31, after both halves
-//               have read their S).  The running max is only moved (and O
-//               rescaled in TMEM, each half its 64 channels, after waiting
-//               for PV_{j-1}) when it grows by more than 2^8; otherwise the
-//               stale max is kept, which is exact because O and the row sum
-//               always use the same max.  Each half keeps its own partial row
-//               sum; the epilogue adds them: O / l -> bf16, lse.
+//               buffer (column t/2 holds elements t, t+1).  A chain's running
+//               max only moves (and its O is rescaled in TMEM, after its
+//               previous PV) when it grows by more than 2^8; a stale max is
+//               exact because the chain's O and row sum use the same one.
+//               Epilogue: the two chains exchange (max, sum) per row through
+//               shared memory; thread (row, chain c) writes channels
+//               64c..64c+63 of O = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / l, and lse.
 // A pre-pass compacts the route into shared memory, skipping ids outside
 // [0, M) and repeats (flagged in dev_status).
 //
@@ -58,26 +55,25 @@ namespace {
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // tokens per KV tile
 constexpr int D = 128;   // head dim
-constexpr int kThreads = 320;  // TMA warp, MMA warp, 8 softmax warps
+constexpr int kThreads = 320;  // TMA warp, MMA warp, 2 x 4 softmax warps
+constexpr int kChainThreads = 128;  // softmax threads of one chain
 constexpr int kSoftThreads = 256;
 constexpr uint32_t kTileBytes = BN * D * 2;      // 32 KB
 constexpr uint32_t kHalfBytes = kTileBytes / 2;  // one 64-channel box
 constexpr int kMaxRoute = VELOX_MAX_ROUTE;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kSBufs = 2;         // S/P buffers in TMEM, columns 0 and 128
-constexpr uint32_t kColQ = 256;   // Q (bf16 pairs, 64 columns)
-constexpr uint32_t kColO = 384;   // O accumulator (fp32, 128 columns)
+constexpr int kSBufs = 2;         // S/P buffers in TMEM (one per chain), columns 0 and 128
+constexpr uint32_t kColO = 256;   // O accumulators (fp32, 128 columns each), 256 and 384
 constexpr int kMaxSlots = 6;      // K/V ring slots of 32 KB
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest tolerated growth
 
 // shared-memory layout (offsets from a 1024-byte aligned base)
-constexpr uint32_t kOffRing = 0;
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffRing = kOffQ + kTileBytes;
 // barriers, misc and the dynamic tail follow the ring (offset set at launch)
-constexpr uint32_t kNumBars = 1 + 2 * kMaxSlots + 3 * kSBufs + 1 + kSBufs + 1;
+// q_full, the K/V ring, s_full/p_full/pv_done per chain, x_fin, mma_done
+constexpr uint32_t kNumBars = 1 + 2 * kMaxSlots + 3 * kSBufs + 1 + 1;
 constexpr uint32_t kMiscBytes = 64;
-// half-row maxima, rounded up to bf16, in two alternating slots ([2][2][128]
-// bf16), then the two partial row sums of the epilogue ([2][128] fp32)
-constexpr uint32_t kXchBytes = 2 * 2 * BM * 2 + 2 * BM * 4;
 constexpr uint32_t kSmemLimit = 227 * 1024;
 
 struct AttnArgs {
@@ -95,7 +91,6 @@ struct AttnArgs {
   int32_t *dev_status;
   int nslot;              // K/V ring slots in use (4..kMaxSlots)
   uint32_t bar_offset;    // byte offset of the barriers from the aligned base
-  uint32_t xch_offset;    // half-row maxima exchange area (bf16 bits)
   uint32_t list_offset;   // route list (uint16)
   uint32_t bits_offset;   // id bitmap (uint32)
 };
@@ -122,39 +117,31 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-// bf16 bits of finite x rounded towards +inf.
-__device__ __forceinline__ uint16_t bf16_round_up(float x) {
-  const uint32_t u = __float_as_uint(x);
-  uint32_t hi = u >> 16;
-  if ((u & 0xffffu) != 0u && (u >> 31) == 0u) hi += 1u;  // positive: away from 0; negative: toward 0
-  return static_cast<uint16_t>(hi);
-}
-
 // Warp-uniform bounded wait (tcgen05.ld/st after it are warp-collective).
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
 }
 
+// 10 warps: three share a scheduler, whose 16 K registers then allow 168 each
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_kernel(const __grid_constant__ CUtensorMap tmK,
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
                 const __grid_constant__ CUtensorMap tmVc, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
+  uint8_t *sQ = base + kOffQ;
   uint8_t *ring = base + kOffRing;
   uint64_t *bar = reinterpret_cast<uint64_t *>(base + a.bar_offset);
   uint64_t *q_full = bar;
-  uint64_t *slot_full = bar + 1;
+  uint64_t *slot_full = q_full + 1;
   uint64_t *slot_empty = slot_full + kMaxSlots;
-  uint64_t *s_full = slot_empty + kMaxSlots;
-  uint64_t *p_full = s_full + kSBufs;
-  uint64_t *pv_done = p_full + kSBufs;
-  uint64_t *mma_done = pv_done + kSBufs;
-  uint64_t *x_max = mma_done + 1;   // both half-row maxima of S buffer b written
-  uint64_t *x_fin = x_max + kSBufs;  // both partial row sums written
+  uint64_t *s_full = slot_empty + kMaxSlots;   // [chain]
+  uint64_t *p_full = s_full + kSBufs;          // [chain]
+  uint64_t *pv_done = p_full + kSBufs;         // [chain]
+  uint64_t *x_fin = pv_done + kSBufs;          // both chains' (max, sum) written
+  uint64_t *mma_done = x_fin + 1;
   uint8_t *misc = base + a.bar_offset + kNumBars * 8;
-  uint16_t *xch = reinterpret_cast<uint16_t *>(base + a.xch_offset);
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(misc);
   int *s_nvalid = reinterpret_cast<int *>(misc + 4);
   volatile int *s_abort = reinterpret_cast<volatile int *>(misc + 8);
@@ -174,19 +161,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- set-up: barriers, TMEM, route compaction
   if (threadIdx.x == 0) {
-    mbar_init(q_full, kSoftThreads);  // Q written to TMEM by the softmax threads
+    mbar_init(q_full, 1);
     for (int s = 0; s < kMaxSlots; ++s) {
       mbar_init(&slot_full[s], 1);
       mbar_init(&slot_empty[s], 1);
     }
     for (int b = 0; b < kSBufs; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], kSoftThreads);
+      mbar_init(&p_full[b], kChainThreads);
       mbar_init(&pv_done[b], 1);
-      mbar_init(&x_max[b], kSoftThreads);
     }
-    mbar_init(mma_done, 1);
     mbar_init(x_fin, kSoftThreads);
+    mbar_init(mma_done, 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -243,12 +229,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ================= TMA producer =================
     if (lane == 0 && n > 0) {
+      prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       if (a.n_cur > 0) {
         prefetch_tmap(&tmKc);
         prefetch_tmap(&tmVc);
       }
+      mbar_arrive_expect_tx(q_full, kTileBytes);
+      tma_load_3d(sQ, &tmQ, q_full, 0, i * BM, h);
+      tma_load_3d(sQ + kHalfBytes, &tmQ, q_full, 64, i * BM, h);
       int issued = 0;
       for (int li = 0; li < 2 * n; ++li) {  // load li: K_{li/2} (even) or V_{li/2} (odd)
         const int s = li % nslot;
@@ -268,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // let the copies already in flight land before the CTA goes away
         // (each wait is bounded by the same time limit)
         volatile int never = 0;
+        mbar_wait(q_full, 0, &never);
         for (int li = issued - nslot < 0 ? 0 : issued - nslot; li < issued; ++li) {
           never = 0;
           mbar_wait(&slot_full[li % nslot], (li / nslot) & 1, &never);
@@ -279,17 +270,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && n > 0) {
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false);
       constexpr uint32_t idPV = idesc_bf16_f32(BM, D, true);
-      const uint32_t ra = smem_u32(ring);
+      const uint32_t qa = smem_u32(sQ), ra = smem_u32(ring);
       auto issue_s = [&](int j) -> bool {
         const int li = 2 * j, s = li % nslot;
         if (!mbar_wait(&slot_full[s], (li / nslot) & 1, s_abort)) return false;
         tc_fence_after();
         const uint32_t ka = ra + s * kTileBytes;
-        const uint32_t sb = tmem + (j % kSBufs) * BN;
+        const uint32_t sb = tmem + (j & 1) * BN;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_bf16_ts(sb, tmem + kColQ + k * 8, kmajor_desc(ka, k), idS, k > 0);
-        tc_commit(&s_full[j % kSBufs]);
+          mma_bf16_ss(sb, kmajor_desc(qa, k), kmajor_desc(ka, k), idS, k > 0);
+        tc_commit(&s_full[j & 1]);
         tc_commit(&slot_empty[s]);
         return true;
       };
@@ -297,8 +288,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = issue_s(0);
       if (ok && n > 1) ok = issue_s(1);
       for (int j = 0; ok && j < n; ++j) {
-        const int b = j % kSBufs;
-        if (!mbar_wait(&p_full[b], (j / kSBufs) & 1, s_abort)) break;
+        const int b = j & 1;  // chain
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(&p_full[b], ph, s_abort)) break;
         const int li = 2 * j + 1, s = li % nslot;
         if (!mbar_wait(&slot_full[s], (li / nslot) & 1, s_abort)) break;
         tc_fence_after();
@@ -306,12 +298,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t pb = tmem + b * BN;  // P_j: first 64 columns of its S buffer
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k)
-          mma_bf16_ts(tmem + kColO, pb + k * 8, vmn_desc(va, k), idPV, (j > 0 || k > 0));
+          mma_bf16_ts(tmem + kColO + b * D, pb + k * 8, vmn_desc(va, k), idPV, (j >= 2 || k > 0));
         tc_commit(&pv_done[b]);
         tc_commit(&slot_empty[s]);
         if (j + 2 < n) {
           // S_{j+2} goes into the buffer P_j occupies: PV_j must be done
-          if (!mbar_wait(&pv_done[b], (j / kSBufs) & 1, s_abort)) break;
+          if (!mbar_wait(&pv_done[b], ph, s_abort)) break;
           if (!issue_s(j + 2)) break;
         }
       }
@@ -323,143 +315,146 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ================= softmax / epilogue (warps 2..9) =================
     const int quarter = warp & 3;
-    const int hf = (warp - 2) >> 2;     // which 64 columns of the row
+    const int ch = (warp - 2) >> 2;     // chain: tiles j with j % 2 == ch
     const int r = quarter * 32 + lane;  // query row within the tile = TMEM lane
     const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t sb = trow + ch * BN;                 // this chain's S buffer
+    const uint32_t ob = trow + kColO + ch * D;          // this chain's O
     const float c = a.scale_log2;
-    float m_run = -INFINITY, l = 0.f;  // l: this half's partial row sum
+    float m_run = -INFINITY, l = 0.f;
     bool ok = true;
-    if (n > 0) {
-      // this thread's half of Q row r into TMEM: bf16 pairs, element 2c in the
-      // low half of column c, as the A operand of S = Q K^T expects
-      const uint4 *qsrc = reinterpret_cast<const uint4 *>(
-          a.Q + (((size_t)h * a.N + i) * BM + r) * D + hf * 64);
-      uint32_t qv[32];
+    int last = -1;  // this chain's last tile
+    for (int j = ch; j < n; j += 2) {
+      const uint32_t ph = (j >> 1) & 1;
+      if (!warp_wait(&s_full[ch], ph, s_abort)) { ok = false; break; }
+      tc_fence_after();
+      // two passes over the S row (the register file holds 168 per thread):
+      // the max, then the exponentials 32 columns at a time
+      float mx[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint4 v = __ldg(qsrc + q);
-        qv[4 * q + 0] = v.x;
-        qv[4 * q + 1] = v.y;
-        qv[4 * q + 2] = v.z;
-        qv[4 * q + 3] = v.w;
+      for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t sv[64];
+        tmem_ld32(sb + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(sb + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          mx[k & 7] = fmax3(mx[k & 7], __uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1]));
       }
-      tmem_st32(trow + kColQ + hf * 32, qv);
-      tmem_wait_st();
-    }
-    tc_fence_before();
-    mbar_arrive(q_full);
-    for (int j = 0; j < n; ++j) {
-      const int b = j % kSBufs;
-      const uint32_t ph = (j / kSBufs) & 1;
-      const uint32_t sb = trow + b * BN;
-      if (!warp_wait(&s_full[b], ph, s_abort)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sv[64];
-      tmem_ld32(sb + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(sb + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      tmem_wait_ld();
-      float mx[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) mx[q] = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < 32; ++k)
-        mx[k & 3] = fmax3(mx[k & 3], __uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1]));
-      // exchange the half maxima, each rounded up to bf16 so that both halves
-      // take the same (slightly larger, hence still exact) max; slot j & 1 is
-      // free again because the partner read it before arriving for tile j - 1.
-      // After this wait both halves have read their S columns, so P may
-      // overwrite columns 0..63 of the buffer.
-      const uint16_t mh = bf16_round_up(fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]));
-      xch[((j & 1) * 2 + hf) * BM + r] = mh;
-      tc_fence_before();
-      mbar_arrive(&x_max[b]);
-      if (!warp_wait(&x_max[b], ph, s_abort)) { ok = false; break; }
-      tc_fence_after();
-      const uint16_t mo = xch[((j & 1) * 2 + (hf ^ 1)) * BM + r];
-      const float mt = fmaxf(__uint_as_float(static_cast<uint32_t>(mh) << 16),
-                             __uint_as_float(static_cast<uint32_t>(mo) << 16));
+      const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                             fmaxf(mx[6], mx[7]));
       const float m_cand = fmaxf(m_run, mt * c);
-      const bool grow = m_cand > m_run + kRescaleThreshold;  // always on the first tile
+      const bool grow = m_cand > m_run + kRescaleThreshold;  // always on the chain's first tile
       const float m_use = grow ? m_cand : m_run;
       const float alpha = fast_exp2(m_run - m_use);  // 1 if kept, 0 on the first tile
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // move O to the new max: PV_{j-1} (and every earlier PV) must be done
-        const int jp = j - 1;
-        if (!warp_wait(&pv_done[jp % kSBufs], (jp / kSBufs) & 1, s_abort)) { ok = false; break; }
+      if (last >= 0 && __any_sync(0xffffffffu, grow)) {
+        // move this chain's O to the new max: its previous PV must be done
+        if (!warp_wait(&pv_done[ch], (last >> 1) & 1, s_abort)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
+        for (int cc = 0; cc < 4; ++cc) {
           uint32_t ov[32];
-          const uint32_t oa = trow + kColO + hf * 64 + cc * 32;
-          tmem_ld32(oa, ov);
+          tmem_ld32(ob + cc * 32, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
-          tmem_st32(oa, ov);
+          tmem_st32(ob + cc * 32, ov);
         }
       }
       // exponentials (arguments and row sum in packed pairs); P_j into the
       // first 64 columns of its S buffer: column t/2 holds elements t, t+1
       uint64_t sum2[2] = {0ull, 0ull};
       const uint64_t c2 = f2pack(c, c), nm2 = f2pack(-m_use, -m_use);
-      uint32_t pk[32];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const uint64_t x2 = ffma2(f2pack(__uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1])),
-                                  c2, nm2);
-        float x0, x1;
-        f2unpack(x2, x0, x1);
-        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-        sum2[k & 1] = fadd2(sum2[k & 1], f2pack(p0, p1));
-        pk[k] = pack_bf16x2(p0, p1);
+      for (int qt = 0; qt < 4; ++qt) {  // S columns 32qt.. -> P columns 16qt.. (already read)
+        uint32_t sv[32];
+        tmem_ld32(sb + qt * 32, sv);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const uint64_t x2 = ffma2(f2pack(__uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1])),
+                                    c2, nm2);
+          float x0, x1;
+          f2unpack(x2, x0, x1);
+          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          sum2[k & 1] = fadd2(sum2[k & 1], f2pack(p0, p1));
+          pk[k] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(sb + qt * 16, pk);
       }
-      tmem_st32(sb + hf * 32, pk);
       float sa, sb2;
       f2unpack(fadd2(sum2[0], sum2[1]), sa, sb2);
       tmem_wait_st();
       l = l * alpha + (sa + sb2);
       m_run = m_use;
+      last = j;
       tc_fence_before();
-      mbar_arrive(&p_full[b]);
+      mbar_arrive(&p_full[ch]);
     }
-    // epilogue: the row sum is the sum of the two halves' partial sums
-    uint16_t *orow = a.O + ((size_t)row * BM + r) * D + hf * 64;
+    // epilogue: merge the two chains.  Both chains' last PVs must be done
+    // before either O is read; (max, sum) per row go through shared memory
+    // (the ring, idle once every PV is done).
     bool have = ok && n > 0;
     if (have) {
-      const int jl = n - 1;
-      have = mbar_wait(&pv_done[jl % kSBufs], (jl / kSBufs) & 1, s_abort);
+      for (int cc = 0; cc < 2 && cc < n; ++cc) {
+        const int lc = ((n - 1) & 1) == cc ? n - 1 : n - 2;  // chain cc's last tile
+        if (!mbar_wait(&pv_done[cc], (lc >> 1) & 1, s_abort)) { have = false; break; }
+      }
     }
-    float *lx = reinterpret_cast<float *>(base + a.xch_offset + 2 * 2 * BM * 2);
-    lx[hf * BM + r] = l;
+    float *xm = reinterpret_cast<float *>(ring);  // [chain][2][128]: max, sum
+    xm[(ch * 2 + 0) * BM + r] = m_run;
+    xm[(ch * 2 + 1) * BM + r] = l;
     mbar_arrive(x_fin);
-    const bool fin = mbar_wait(x_fin, 0, s_abort);
-    const float l_row = l + lx[(hf ^ 1) * BM + r];
+    const bool fin_ok = mbar_wait(x_fin, 0, s_abort);
+    const float mo = xm[((ch ^ 1) * 2 + 0) * BM + r];
+    const float lo = xm[((ch ^ 1) * 2 + 1) * BM + r];
+    const float m0 = ch == 0 ? m_run : mo, m1 = ch == 0 ? mo : m_run;
+    const float l0 = ch == 0 ? l : lo, l1 = ch == 0 ? lo : l;
+    const float mm = fmaxf(m0, m1);
+    // a chain without tiles has max -inf and sum 0: weight 0, O never read
+    const float w0 = n > 0 ? fast_exp2(m0 - mm) : 0.f;
+    const float w1 = n > 1 ? fast_exp2(m1 - mm) : 0.f;
+    const float l_row = l0 * w0 + l1 * w1;
     // tcgen05.ld is warp-collective: decide once for the whole warp
-    const bool good = __all_sync(0xffffffffu, have && fin && !*s_abort);
+    const bool good = __all_sync(0xffffffffu, have && fin_ok && !*s_abort);
     tc_fence_after();
     const float inv = good ? 1.0f / l_row : 0.f;
+    uint16_t *orow = a.O + ((size_t)row * BM + r) * D + ch * 64;
 #pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      uint32_t ov[32];
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t o0[16], o1[16];
       if (good) {
-        tmem_ld32(trow + kColO + hf * 64 + cc * 32, ov);
+        tmem_ld16(trow + kColO + ch * 64 + cc * 16, o0);
+        if (n > 1) tmem_ld16(trow + kColO + D + ch * 64 + cc * 16, o1);
         tmem_wait_ld();
       } else {
 #pragma unroll
-        for (int k = 0; k < 32; ++k) ov[k] = 0u;
+        for (int k = 0; k < 16; ++k) o0[k] = 0u;
       }
+      if (!good || n < 2) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 v;
-        v.x = pack_bf16x2(__uint_as_float(ov[8 * q + 0]) * inv, __uint_as_float(ov[8 * q + 1]) * inv);
-        v.y = pack_bf16x2(__uint_as_float(ov[8 * q + 2]) * inv, __uint_as_float(ov[8 * q + 3]) * inv);
-        v.z = pack_bf16x2(__uint_as_float(ov[8 * q + 4]) * inv, __uint_as_float(ov[8 * q + 5]) * inv);
-        v.w = pack_bf16x2(__uint_as_float(ov[8 * q + 6]) * inv, __uint_as_float(ov[8 * q + 7]) * inv);
-        *reinterpret_cast<uint4 *>(orow + cc * 32 + q * 8) = v;
+        for (int k = 0; k < 16; ++k) o1[k] = 0u;
+      }
+      const float s0 = w0 * inv, s1 = w1 * inv;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          v[e] = __uint_as_float(o0[8 * q + e]) * s0 + __uint_as_float(o1[8 * q + e]) * s1;
+        uint4 u;
+        u.x = pack_bf16x2(v[0], v[1]);
+        u.y = pack_bf16x2(v[2], v[3]);
+        u.z = pack_bf16x2(v[4], v[5]);
+        u.w = pack_bf16x2(v[6], v[7]);
+        *reinterpret_cast<uint4 *>(orow + cc * 16 + q * 8) = u;
       }
     }
-    if (a.lse && hf == 0)
-      a.lse[(size_t)row * BM + r] = good ? (m_run + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
+    if (a.lse && ch == 0)
+      a.lse[(size_t)row * BM + r] = good ? (mm + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
   }
 
   if (*s_abort && threadIdx.x == 0) flag_error(a.dev_status, VELOX_DEV_WAIT_TIMEOUT);
@@ -511,9 +506,9 @@ cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                         float softmax_scale, uint16_t *O, float *lse, int32_t *dev_status,
                         cudaStream_t stream, bool *map_failed) {
   *map_failed = false;
-  CUtensorMap mk, mv, mkc, mvc;
+  CUtensorMap mq, mk, mv, mkc, mvc;
   const bool cur = K_cur != nullptr && N_cur > 0;
-  if (!make_map(&mk, K, M * BN, H) ||
+  if (!make_map(&mq, Q, N * BM, H) || !make_map(&mk, K, M * BN, H) ||
       !make_map(&mv, V, M * BN, H) ||
       !make_map(&mkc, cur ? K_cur : K, cur ? N_cur * BN : M * BN, H) ||
       !make_map(&mvc, cur ? V_cur : V, cur ? N_cur * BN : M * BN, H)) {
@@ -537,7 +532,7 @@ cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
   // tail after the ring: barriers, misc, route list (uint16), id bitmap
   const uint32_t list_bytes = route_ids ? ((uint32_t)R_max * 2u + 15u) & ~15u : 0u;
   const uint32_t bits_bytes = route_ids ? (uint32_t)((M + 31) / 32) * 4u : 0u;
-  const uint32_t tail = kNumBars * 8 + kMiscBytes + kXchBytes + list_bytes + bits_bytes;
+  const uint32_t tail = kNumBars * 8 + kMiscBytes + list_bytes + bits_bytes;
   int nslot = kMaxSlots;
   while (nslot > 4 && kOffRing + nslot * kTileBytes + tail + 1024 > kSmemLimit) --nslot;
   // loads go K_0, V_0, K_1, V_1, ... round the ring; load li reuses the slot
@@ -546,15 +541,14 @@ cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
   nslot &= ~1;
   a.nslot = nslot;
   a.bar_offset = kOffRing + nslot * kTileBytes;
-  a.xch_offset = a.bar_offset + kNumBars * 8 + kMiscBytes;
-  a.list_offset = a.xch_offset + kXchBytes;
+  a.list_offset = a.bar_offset + kNumBars * 8 + kMiscBytes;
   a.bits_offset = a.list_offset + list_bytes;
   const size_t smem = (size_t)a.bits_offset + bits_bytes + 1024;  // + alignment slack
   if (smem > kSmemLimit) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  attn_kernel<<<H * N, kThreads, smem, stream>>>(mk, mv, mkc, mvc, a);
+  attn_kernel<<<H * N, kThreads, smem, stream>>>(mq, mk, mv, mkc, mvc, a);
   return cudaGetLastError();
 }
 

@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(RouteArgs a) {
   __shared__ double s_dred[kWarps];
   __shared__ int s_ired[kWarps];
   __shared__ int s_hist[256];
-  __shared__ int s_digit, s_greater, s_ntake;
+  __shared__ int s_digit, s_greater, s_equal, s_ntake;
 
   const int row = blockIdx.x;
   const int i = row % a.N;
@@ -192,7 +192,11 @@ __global__ void __launch_bounds__(kThreads) route_kernel(RouteArgs a) {
         int run = incl - lt;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          if (run < need && run + c[j] >= need) { s_digit = 255 - 8 * tid - j; s_greater = run; }
+          if (run < need && run + c[j] >= need) {
+            s_digit = 255 - 8 * tid - j;
+            s_greater = run;
+            s_equal = c[j];
+          }
           run += c[j];
         }
       }
@@ -200,10 +204,16 @@ __global__ void __launch_bounds__(kThreads) route_kernel(RouteArgs a) {
       prefix |= static_cast<uint64_t>(s_digit) << shift;
       mask |= 0xFFull << shift;
       need -= s_greater;
+      const bool all_of_digit = (need == s_equal);
       __syncthreads();
+      // every key that shares the prefix so far is taken: the lower bytes
+      // cannot change the selection
+      if (all_of_digit) break;
     }
   }
-  // prefix = key of the k_sel-th largest; `need` ties at that key are taken.
+  // keys are compared on their bytes under `mask`: prefix = those bytes of
+  // the k_sel-th largest; `need` keys equal to it there are taken, lowest
+  // ids first.
 
   // ---- compaction in id order (thread t owns ids [t*c, t*c + c))
   const int chunk = (M + kThreads - 1) / kThreads;
@@ -213,7 +223,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(RouteArgs a) {
     for (int r = lo; r < hi; ++r) {
       if (r >= pb && r < pe) continue;
       if (select_all) { ++n_gt; continue; }
-      const uint64_t u = order_key(keys[r]);
+      const uint64_t u = order_key(keys[r]) & mask;
       n_gt += (u > prefix);
       n_tie += (u == prefix);
     }
@@ -232,7 +242,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(RouteArgs a) {
       if (select_all) {
         inc = true;
       } else {
-        const uint64_t u = order_key(keys[r]);
+        const uint64_t u = order_key(keys[r]) & mask;
         inc = (u > prefix) || (u == prefix && ties_seen++ < take_tie);
       }
       if (inc && pos < a.kcap) {
