@@ -14,7 +14,8 @@
 //                         warp then counts the G^3 cell centres of the query
 //                         box inside the history box for each candidate of
 //                         its 32 together.
-//   coverage_kernel       one CTA per query block: every token's warped depth
+//   coverage_kernel       a cluster of 4 CTAs per query block, each taking a
+//                         quarter of its tokens: every token's warped depth
 //                         is back-projected and tested against the past slabs
 //                         (rectangle and depth range in the slab's camera);
 //                         rho = covered tokens / b, covered = rho >= eta.
@@ -22,12 +23,17 @@
 //                         the block's token cloud are dropped first (with a
 //                         margin far above rounding, so no decision changes);
 //                         a token's projection into a camera is formed once
-//                         for a run of slabs of that camera.
+//                         for a run of slabs of that camera; the quarters'
+//                         covered counts meet in CTA 0's shared memory.
 //
 // Every inside/outside decision uses explicitly rounded fp32 operations
 // (__fmul_rn, __fadd_rn, __fsub_rn, __fdiv_rn) in a fixed order, so no
 // contraction into FMA changes which side of a face a point lands on.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace velox {
 namespace {
@@ -220,10 +226,12 @@ __global__ void __launch_bounds__(256) slab_overlap_kernel(const velox_camera *_
   if (r < M) g[(size_t)i * M + r] = out;
 }
 
-// One CTA per query block, b * kParts working threads (the block rounded up
-// to whole warps): thread (t, part) tests token t against the part-th
-// contiguous share of the surviving slabs.
-constexpr int kParts = 8;
+// A cluster of kSplit CTAs per query block; CTA q takes tokens
+// [q tpc, (q + 1) tpc) with tpc = ceil(b / kSplit), and tpc * kParts working
+// threads (rounded up to whole warps): thread (t, part) tests token t against
+// the part-th contiguous share of the surviving slabs.
+constexpr int kSplit = 4;
+constexpr int kParts = 32;
 constexpr int kSlabChunk = 2048;  // slabs culled and tested per round
 
 // World corner k (bit 0: u, bit 1: v, bit 2: depth) of a slab's frustum.
@@ -235,25 +243,32 @@ __device__ __forceinline__ void frustum_corner(const velox_camera &c, const velo
   cam_to_world(c.R, c.C, x, X);
 }
 
-__global__ void __launch_bounds__(1024) coverage_kernel(const velox_camera *__restrict__ cams, int n_cams,
+__global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(1024)
+    coverage_kernel(const velox_camera *__restrict__ cams, int n_cams,
                                 const velox_slab *__restrict__ qs, const float *__restrict__ q_uvz,
                                 int b, const velox_slab *__restrict__ hs, int M, float eta,
                                 float *__restrict__ rho, uint8_t *__restrict__ covered,
                                 int32_t *dev_status) {
   extern __shared__ int s_cov_raw[];
-  volatile int *s_cov = s_cov_raw;  // [b] per-token covered flags (read by other parts)
+  volatile int *s_cov = s_cov_raw;  // [tpc] per-token covered flags (read by other parts)
   __shared__ int s_list[kSlabChunk];
   __shared__ int s_nlist;
   __shared__ float s_red[32][4];
   __shared__ float s_sphere[4];  // token cloud centre and radius
-  const int i = blockIdx.x;
-  const int t = threadIdx.x % b, part = threadIdx.x / b;
-  const bool act = part < kParts;
+  __shared__ int s_total;        // CTA 0 of the cluster: covered tokens of the block
+  cg::cluster_group cluster = cg::this_cluster();
+  const int q = (int)cluster.block_rank();
+  const int i = blockIdx.x / kSplit;
+  const int tpc = (b + kSplit - 1) / kSplit;
+  const int tl = threadIdx.x % tpc, part = threadIdx.x / tpc;
+  const int t = q * tpc + tl;  // token of the block
+  const bool act = part < kParts && t < b;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  for (int k = threadIdx.x; k < b; k += blockDim.x) s_cov[k] = 0;
+  for (int k = threadIdx.x; k < tpc; k += blockDim.x) s_cov[k] = 0;
+  if (threadIdx.x == 0) s_total = 0;
   const velox_slab sq = qs[i];
   const bool q_ok = sq.cam >= 0 && sq.cam < n_cams;
-  if (!q_ok && threadIdx.x == 0) flag_error(dev_status, VELOX_DEV_BAD_CAMERA);
+  if (!q_ok && threadIdx.x == 0 && q == 0) flag_error(dev_status, VELOX_DEV_BAD_CAMERA);
   float X[3] = {0.f, 0.f, 0.f};
   bool live = false;
   if (q_ok && act) {
@@ -367,7 +382,7 @@ __global__ void __launch_bounds__(1024) coverage_kernel(const velox_camera *__re
       bool front = false;
       float pu = 0.f, pv = 0.f, dz = 0.f;
       for (int k = part * per; k < k1; ++k) {
-        if (s_cov[t]) break;  // another part already covered this token
+        if (s_cov[tl]) break;  // another part already covered this token
         const velox_slab sr = hs[s_list[k]];
         if (sr.cam != last_cam) {
           last_cam = sr.cam;
@@ -383,23 +398,27 @@ __global__ void __launch_bounds__(1024) coverage_kernel(const velox_camera *__re
         }
         if (front && sr.zlo <= dz && dz <= sr.zhi && sr.u0 <= pu && pu < sr.u1 && sr.v0 <= pv &&
             pv < sr.v1) {
-          s_cov[t] = 1;
+          s_cov[tl] = 1;
           break;
         }
       }
     }
     __syncthreads();
   }
+  // every CTA's s_total is initialised before any CTA adds to CTA 0's
+  cluster.sync();
   if (threadIdx.x < 32) {
     int n = 0;
-    for (int k = threadIdx.x; k < b; k += 32) n += s_cov[k];
+    for (int k = threadIdx.x; k < tpc; k += 32) n += s_cov[k];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) n += __shfl_xor_sync(0xffffffffu, n, off);
-    if (threadIdx.x == 0) {
-      const float rh = (float)n / (float)b;
-      rho[i] = rh;
-      covered[i] = rh >= eta ? 1 : 0;
-    }
+    if (threadIdx.x == 0) atomicAdd(cluster.map_shared_rank(&s_total, 0), n);
+  }
+  cluster.sync();
+  if (q == 0 && threadIdx.x == 0) {
+    const float rh = (float)s_total / (float)b;
+    rho[i] = rh;
+    covered[i] = rh >= eta ? 1 : 0;
   }
 }
 
@@ -417,9 +436,11 @@ cudaError_t launch_coverage(const velox_camera *cams, int n_cams, const velox_sl
                             const float *q_uvz, int N, int b, const velox_slab *hs, int M,
                             float eta, float *rho, uint8_t *covered, int32_t *dev_status,
                             cudaStream_t stream) {
-  const int threads = (b * kParts + 31) / 32 * 32;
-  coverage_kernel<<<N, threads, b * sizeof(int), stream>>>(cams, n_cams, qs, q_uvz, b, hs, M, eta,
-                                                           rho, covered, dev_status);
+  const int tpc = (b + kSplit - 1) / kSplit;
+  const int threads = (tpc * kParts + 31) / 32 * 32;
+  coverage_kernel<<<N * kSplit, threads, tpc * sizeof(int), stream>>>(cams, n_cams, qs, q_uvz, b,
+                                                                      hs, M, eta, rho, covered,
+                                                                      dev_status);
   return cudaGetLastError();
 }
 
