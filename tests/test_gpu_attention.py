@@ -178,3 +178,21 @@ def test_large_logits_stay_finite(lib):
     O, lse, st = _attend(inp, rid, rlen, M)
     ref = attention_rows(inp.Q, inp.K, inp.V, sorted(routes), lambda h, i: routes[(h, i)])
     assert_attention_close(O, lse, ref)
+
+
+def test_longest_route_the_abi_allows(lib):
+    # R_max = VELOX_MAX_ROUTE (4096): row 0 visits all 4096 tiles (= dense),
+    # row 1 a ragged random 1500, row 2 a single tile
+    H, N, M = 1, 3, 4096
+    wl = small(H, N, M, 0)
+    inp = make_inputs(wl, "cuda")
+    r = np.random.default_rng(17)
+    routes = {(0, 0): list(range(M)),
+              (0, 1): sorted(r.choice(M, size=1500, replace=False).tolist()),
+              (0, 2): [int(r.integers(M))]}
+    R_max = 4096
+    rid, rlen = _routes_tensor(routes, H, N, R_max)
+    O, lse, st = _attend(inp, rid, rlen, R_max)
+    assert st == 0
+    ref = attention_rows(inp.Q, inp.K, inp.V, sorted(routes), lambda h, i: routes[(h, i)])
+    assert_attention_close(O, lse, ref)

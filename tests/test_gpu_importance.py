@@ -64,3 +64,20 @@ def test_importance_peaked_logits(lib):
     for h, ph in ref.items():
         g = f64(p[h])
         assert np.all(np.abs(g - ph) <= 50 * P_RTOL * ph + 1e-30)
+
+
+def test_importance_at_the_largest_history(lib):
+    # M = VELOX_MAX_BLOCKS (65536): p of one row, checked where the oracle
+    # can afford it -- the row sums to 1, and sampled pairs of blocks have
+    # the fp64 ratio p_r / p_s = exp(l_r - l_s) of their own mean keys
+    H, N, M = 1, 1, 65536
+    inp = make_inputs(small(H, N, M, 0), "cuda")
+    p = f64(_run(lib, inp, 1.0)[0, 0])
+    assert np.all(np.isfinite(p)) and abs(p.sum() - 1.0) < 1e-4
+    qbar = f64(inp.Q[0, :128]).mean(axis=0)
+    r = np.random.default_rng(5)
+    ids = r.choice(M, size=24, replace=False)
+    kbar = {int(b): f64(inp.K[0, b * 128:(b + 1) * 128]).mean(axis=0) for b in ids}
+    for a_, b_ in zip(ids[::2], ids[1::2]):
+        ratio = math.exp(float(qbar @ kbar[int(a_)] - qbar @ kbar[int(b_)]))
+        assert abs(p[a_] / p[b_] / ratio - 1.0) <= 2 * P_RTOL
