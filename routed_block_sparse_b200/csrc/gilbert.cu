@@ -145,12 +145,13 @@ __global__ void order_kernel(Lattice L, int n_cells, int32_t *rank_of_cell,
 // inverse are built once in shared memory and every lookup is a table read;
 // otherwise each lookup descends the recursion.
 constexpr int kFrameSmemCells = 8192;
+constexpr int kNbrThreads = 512;
 
 __global__ void neighbour_kernel(Lattice L, int q_chunk, int cache_first, int n_cache,
                                  int32_t *nbr_ids, int32_t *nbr_cnt, int S_max, int use_table,
                                  int32_t *dev_status) {
   extern __shared__ int smem_i[];
-  __shared__ int s_scan[256];
+  __shared__ int s_scan[kNbrThreads];
   const int HW = L.HW();
   int *r2 = smem_i;                             // [HW] when use_table
   int *inv = smem_i + (use_table ? HW : 0);     // [HW] when use_table
@@ -270,7 +271,7 @@ cudaError_t launch_gilbert(int T, int H, int W, int n_chunks, int b, int q_chunk
                                            (int)smem);
       if (e != cudaSuccess) return e;
     }
-    neighbour_kernel<<<per_chunk, 256, smem, stream>>>(L, q_chunk, cache_first, n_cache,
+    neighbour_kernel<<<per_chunk, kNbrThreads, smem, stream>>>(L, q_chunk, cache_first, n_cache,
                                                        nbr_ids, nbr_cnt, S_max, use_table,
                                                        dev_status);
     return cudaGetLastError();
