@@ -25,9 +25,11 @@
 //               memory) and, as soon as that has completed, S_{j+2} into the
 //               same buffer.
 //   warps 2-5   softmax of the even tiles, warps 6-9 of the odd tiles: one
-//               query row per thread (its TMEM lane).  One TMEM read of the S
-//               row, a three-input max, scaled exponent arguments and the
-//               row sum in packed fp32x2 arithmetic, exponentials on MUFU,
+//               query row per thread (its TMEM lane).  Two TMEM reads of the
+//               S row (168 registers per thread do not hold the row and the
+//               rest): the three-input max, then 32 columns at a time the
+//               scaled exponent arguments and the row sum in packed fp32x2
+//               arithmetic, exponentials on MUFU,
 //               P_j packed to bf16 into the first 64 columns of its own S
 //               buffer (column t/2 holds elements t, t+1).  A chain's running
 //               max only moves (and its O is rescaled in TMEM, after its
@@ -41,8 +43,8 @@
 //
 // Two-phase form (digest, "Reproducibility": the two-phase tile loop): after
 // the routed history tiles the same loop visits the n_cur tiles of the
-// current chunk's own K/V (separate tensors), under the same online softmax,
-// so one normaliser covers both phases.
+// current chunk's own K/V (separate tensors), alternating between the two
+// chains like any other tiles, so the merged normaliser covers both phases.
 #include <cudaTypedefs.h>
 
 #include <mutex>
