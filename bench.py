@@ -161,13 +161,14 @@ def aggregate(flops_step: float, ms_step: float, world: int, device="cuda"):
 
 
 # ---------------------------------------------------------------- oracle ---
-def cpu_oracle_sample(inp, attn_rows: int = 48, heads=(0, 1, 2, 3)):
+def cpu_oracle_sample(inp, attn_rows: int = 48, heads=(0, 1, 2, 3), step_heads=None):
     """Time the oracle on a bounded sample of one step and scale to a step.
 
     Sample: the neighbour table, importance of `heads` (all 48 x 2256 blocks
     each), the routes of their rows, and attention of `attn_rows` rows of
     the first of them.  The step estimate multiplies each part by its share
-    of the full step (40 heads, 1920 rows).
+    of the full step (`step_heads` heads, default the workload's, and their
+    rows).
     """
     from oracle import attention as oatt
     from oracle import gilbert as ogil
@@ -177,6 +178,8 @@ def cpu_oracle_sample(inp, attn_rows: int = 48, heads=(0, 1, 2, 3)):
 
     wl = inp.wl
     H, N, M, b = wl.heads, wl.n_q_blocks, wl.n_kv_blocks, wl.b
+    if step_heads is not None:
+        H = step_heads
     prm = ort.Params(lam=wl.params.lam, tau=wl.params.tau, g_ref=wl.params.g_ref,
                      theta_cov=wl.params.theta_cov, theta_unc=wl.params.theta_unc,
                      k_cov=wl.params.k_cov, k_unc=wl.params.k_unc)
@@ -218,13 +221,16 @@ def run_reference(args, world, rank):
     """--impl reference: the CPU oracle, on the host cores, rank 0 only."""
     if rank != 0:
         return
+    import dataclasses
     from synth import config, make_inputs
     wl = config(3)
-    inp = make_inputs(wl, "cpu")
+    # the sample works on one head: draw a one-head layer of the same shape
+    # and distributions (drawing all 40 heads on the CPU would take minutes)
+    inp = make_inputs(dataclasses.replace(wl, heads=1), "cpu")
     # FLOPs of the step: mean route length of the sampled head's oracle routes
     times, flops_step = [], None
     for s in range(args.warmup + args.steps):
-        r = cpu_oracle_sample(inp, attn_rows=8, heads=(0,))
+        r = cpu_oracle_sample(inp, attn_rows=8, heads=(0,), step_heads=wl.heads)
         if s >= args.warmup:
             times.append(r["step_s"])
         if flops_step is None:
