@@ -108,7 +108,7 @@ typedef struct {
 /* Human-readable text of a status; never NULL. */
 VELOX_API const char *velox_status_string(velox_status s);
 
-/* ABI version of this header (major * 100 + minor): 101. */
+/* ABI version of this header (major * 100 + minor): 102. */
 VELOX_API int velox_abi_version(void);
 
 /*

@@ -114,7 +114,7 @@ const char *velox_status_string(velox_status s) {
   return "unknown status";
 }
 
-int velox_abi_version(void) { return 101; }
+int velox_abi_version(void) { return 102; }
 
 }  // extern "C"
 

@@ -60,7 +60,7 @@ def test_binding_names_match_header(built):
 
 def test_status_strings_and_version(built):
     import routed_block_sparse_b200 as rbs
-    assert rbs.velox_abi_version() == 101
+    assert rbs.velox_abi_version() == 102
     for s in range(8):
         assert isinstance(rbs.velox_status_string(s), str) and rbs.velox_status_string(s)
     assert rbs.velox_status_string(99) == "unknown status"
