@@ -269,23 +269,24 @@ def run_velox(args, world, rank, local):
     T, Hl, Wl = wl.lattice
     stream = torch.cuda.current_stream(dev)
 
-    def step(ev=None):
+    def step(ev=None, st=None):
+        st = stream if st is None else st
         if ev is not None:
-            ev[0].record(stream)
+            ev[0].record(st)
         rbs.velox_gilbert_order(T, Hl, Wl, wl.n_chunks, b, wl.q_chunk, wl.cache_first_block, M,
                                 nbr_ids=layer.nbr_ids, nbr_cnt=layer.nbr_cnt,
-                                S_max=layer.S_max, dev_status=layer.dev_status, stream=stream)
+                                S_max=layer.S_max, dev_status=layer.dev_status, stream=st)
         if ev is not None:
-            ev[1].record(stream)
-        layer.importance(inp.Q, inp.K, stream)
+            ev[1].record(st)
+        layer.importance(inp.Q, inp.K, st)
         if ev is not None:
-            ev[2].record(stream)
-        layer.route(inp.g, inp.covered, stream=stream)
+            ev[2].record(st)
+        layer.route(inp.g, inp.covered, stream=st)
         if ev is not None:
-            ev[3].record(stream)
-        layer.attend(inp.Q, inp.K, inp.V, stream=stream)
+            ev[3].record(st)
+        layer.attend(inp.Q, inp.K, inp.V, stream=st)
         if ev is not None:
-            ev[4].record(stream)
+            ev[4].record(st)
 
     for _ in range(args.warmup):
         step()
@@ -359,6 +360,10 @@ def run_velox(args, world, rank, local):
         "clocks": clocks.summary(),
     }
 
+    # the same step captured once as a CUDA graph and replayed (the seven
+    # launches go out as one graph launch); reported beside the eager timing
+    line["graph"] = _graph_replay(step, args.steps, dev)
+
     # end to end through the public API with host buffers
     if args.e2e_steps > 0:
         line["e2e"] = _e2e(args, wl, inp, layer, dev, stream, flops_step, world)
@@ -369,6 +374,28 @@ def run_velox(args, world, rank, local):
                                 "sample_seconds": r["sample_s"]}
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def _graph_replay(step, steps, dev):
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step(st=torch.cuda.current_stream(dev))
+        for _ in range(3):
+            graph.replay()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record()
+        for _ in range(steps):
+            graph.replay()
+        b.record()
+        torch.cuda.synchronize(dev)
+        ms = a.elapsed_time(b) / steps
+        del graph
+        return {"ms_per_step": ms, "steps": steps}
+    except Exception as e:  # reported, not fatal: the eager numbers stand alone
+        return {"error": str(e)[:200]}
 
 
 def _e2e(args, wl, inp, layer, dev, stream, flops_step, world):

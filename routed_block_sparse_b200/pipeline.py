@@ -99,6 +99,24 @@ class RoutedLayer:
         self.route(g, covered, stream=stream)
         return self.attend(Q, K, V, stream=stream)
 
+    def capture(self, Q, K, V, g, covered) -> "torch.cuda.CUDAGraph":
+        """Record forward() on these tensors as a CUDA graph.
+
+        Every call of the layer enqueues its kernels on the current stream
+        and allocates nothing, so the four steps (importance, route build,
+        schedule, attention: six kernels) can be captured once and replayed
+        with graph.replay() for as long as the tensors stay in place (new
+        values may be copied into them between replays).  One warm-up call
+        before the capture sets the kernels' shared-memory attributes and
+        builds the tensor maps outside it.
+        """
+        self.forward(Q, K, V, g, covered)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.forward(Q, K, V, g, covered)
+        return graph
+
     def status(self) -> int:
         return int(self.dev_status.item())
 
