@@ -36,30 +36,37 @@ __device__ __forceinline__ bool contains(const Rect &r, int cx, int cy) {
   return i >= 0 && i < iabs(r.ax + r.ay) && j >= 0 && j < iabs(r.bx + r.by);
 }
 
-// The pieces of one recursion level.  Returns the number of pieces (2 or 3)
-// or 0 for a one-cell-thick rectangle (a straight line).
-__device__ __forceinline__ int split(const Rect &r, Rect (&p)[3]) {
-  int nmaj = iabs(r.ax + r.ay), nmin = iabs(r.bx + r.by);
+__device__ __forceinline__ int area(const Rect &r) {
+  return iabs(r.ax + r.ay) * iabs(r.bx + r.by);
+}
+
+// One recursion level: a rectangle is cut across its major edge into two
+// halves (long rectangles) or into three pieces (the near half of the minor
+// edge with the edges swapped, the full-length remainder, and a mirrored piece
+// returning along the far side); halves are made even when the edge is longer
+// than 2.  piece(r, q) builds piece q of r; pieces(r) is their number, 0 for a
+// one-cell-thick rectangle (a straight line).  No arrays: the descent keeps
+// everything in registers.
+__device__ __forceinline__ int pieces(const Rect &r) {
+  const int nmaj = iabs(r.ax + r.ay), nmin = iabs(r.bx + r.by);
   if (nmin == 1 || nmaj == 1) return 0;
-  int ux = sgn(r.ax), uy = sgn(r.ay), vx = sgn(r.bx), vy = sgn(r.by);
+  return 2 * nmaj > 3 * nmin ? 2 : 3;
+}
+__device__ __forceinline__ Rect piece(const Rect &r, int q) {
+  const int nmaj = iabs(r.ax + r.ay), nmin = iabs(r.bx + r.by);
+  const int ux = sgn(r.ax), uy = sgn(r.ay), vx = sgn(r.bx), vy = sgn(r.by);
   int hax = floor_half(r.ax), hay = floor_half(r.ay);
   int hbx = floor_half(r.bx), hby = floor_half(r.by);
   if (2 * nmaj > 3 * nmin) {
     if ((iabs(hax + hay) & 1) && nmaj > 2) { hax += ux; hay += uy; }
-    p[0] = {r.x, r.y, hax, hay, r.bx, r.by};
-    p[1] = {r.x + hax, r.y + hay, r.ax - hax, r.ay - hay, r.bx, r.by};
-    return 2;
+    if (q == 0) return {r.x, r.y, hax, hay, r.bx, r.by};
+    return {r.x + hax, r.y + hay, r.ax - hax, r.ay - hay, r.bx, r.by};
   }
   if ((iabs(hbx + hby) & 1) && nmin > 2) { hbx += vx; hby += vy; }
-  p[0] = {r.x, r.y, hbx, hby, hax, hay};
-  p[1] = {r.x + hbx, r.y + hby, r.ax, r.ay, r.bx - hbx, r.by - hby};
-  p[2] = {r.x + (r.ax - ux) + (hbx - vx), r.y + (r.ay - uy) + (hby - vy), -hbx, -hby,
+  if (q == 0) return {r.x, r.y, hbx, hby, hax, hay};
+  if (q == 1) return {r.x + hbx, r.y + hby, r.ax, r.ay, r.bx - hbx, r.by - hby};
+  return {r.x + (r.ax - ux) + (hbx - vx), r.y + (r.ay - uy) + (hby - vy), -hbx, -hby,
           -(r.ax - hax), -(r.ay - hay)};
-  return 3;
-}
-
-__device__ __forceinline__ int area(const Rect &r) {
-  return iabs(r.ax + r.ay) * iabs(r.bx + r.by);
 }
 
 // Position of cell (cx, cy) on the curve of a W x H frame (W >= H).
@@ -67,20 +74,20 @@ __device__ int frame_rank(int W, int H, int cx, int cy) {
   Rect r = {0, 0, W, 0, 0, H};
   int base = 0;
   for (;;) {
-    Rect p[3];
-    int n = split(r, p);
+    const int n = pieces(r);
     if (n == 0) {
       // a line: along the major edge if it is one cell thick, else the minor
       if (iabs(r.bx + r.by) == 1)
         return base + (cx - r.x) * sgn(r.ax) + (cy - r.y) * sgn(r.ay);
       return base + (cx - r.x) * sgn(r.bx) + (cy - r.y) * sgn(r.by);
     }
-    int k = 0;
-    while (k < n - 1 && !contains(p[k], cx, cy)) {
-      base += area(p[k]);
-      ++k;
+    Rect p = piece(r, 0);
+    int q = 0;
+    while (q < n - 1 && !contains(p, cx, cy)) {
+      base += area(p);
+      p = piece(r, ++q);
     }
-    r = p[k];
+    r = p;
   }
 }
 
@@ -88,8 +95,7 @@ __device__ int frame_rank(int W, int H, int cx, int cy) {
 __device__ void frame_cell(int W, int H, int k, int &cx, int &cy) {
   Rect r = {0, 0, W, 0, 0, H};
   for (;;) {
-    Rect p[3];
-    int n = split(r, p);
+    const int n = pieces(r);
     if (n == 0) {
       if (iabs(r.bx + r.by) == 1) {
         cx = r.x + k * sgn(r.ax);
@@ -100,12 +106,13 @@ __device__ void frame_cell(int W, int H, int k, int &cx, int &cy) {
       }
       return;
     }
+    Rect p = piece(r, 0);
     int q = 0;
-    while (q < n - 1 && k >= area(p[q])) {
-      k -= area(p[q]);
-      ++q;
+    while (q < n - 1 && k >= area(p)) {
+      k -= area(p);
+      p = piece(r, ++q);
     }
-    r = p[q];
+    r = p;
   }
 }
 
