@@ -607,15 +607,16 @@ def run_two_phase(args):
 
 
 def run_variants(args):
-    """The comparison rows, one JSON line each (not the bench line):
-    the geometry-model audit at the audit scale (config 2), the model-only
-    route (lambda = 0) against the fused route at the chunk-48 shape, and the
-    THW-linear order's neighbour table against the Gilbert order's."""
+    """The comparison rows, one JSON line each (not the bench line): the
+    geometry-model audit at the audit scale (40 heads, 12 query blocks, 143
+    history blocks), the model-only route (lambda = 0) against the fused
+    route at the chunk-48 shape, and the THW-linear order's neighbour table
+    against the Gilbert order's."""
     import routed_block_sparse_b200 as rbs
     from routed_block_sparse_b200.pipeline import audit_metrics, layer_for
     from synth import config, make_inputs
 
-    # 1. audit (config 2: H 40, N 12, M 143; tau 0.1, lambda 2, g_ref 0.2)
+    # 1. audit workload (H 40, N 12, M 143; tau 0.1, lambda 2, g_ref 0.2)
     wl = config(2)
     inp = make_inputs(wl, "cuda")
     layer = layer_for(wl)

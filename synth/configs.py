@@ -34,7 +34,7 @@ class Workload:
     """One synthetic problem instance (one layer of one attention call)."""
 
     name: str
-    index: int                    # 1-based config number, enters the seed
+    index: int                    # 1-based workload number, enters the seed
     heads: int
     n_q_blocks: int               # N
     n_kv_blocks: int              # M (history blocks in the cache)
@@ -100,7 +100,8 @@ def sweep_workload(M: int) -> Workload:
 
 
 def config(i: int, layer: int = 0) -> Workload:
-    """Config 5 is config 3 with per-layer seeds (one Workload per layer)."""
+    """Workload i (1-5); workload 5 is the chunk-48 layer with per-layer seeds
+    (one Workload per layer)."""
     if i == 5:
         return replace(CONFIGS[3], index=5, name="chunk48_layers", layer=layer)
     return CONFIGS[i].with_layer(layer)

@@ -93,7 +93,7 @@ def test_pipeline_sweep_and_dense(lib):
 
 @pytest.mark.slow
 def test_pipeline_forty_layers_routes(lib):
-    # config 5: per-layer seeds into reused buffers; routes of two layers and
+    # the 40-layer workload: per-layer seeds into reused buffers; routes of two layers and
     # attention rows of one checked (the oracle is the slow side)
     wl0 = config(5, 0)
     layer = layer_for(wl0)
