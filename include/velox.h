@@ -108,7 +108,7 @@ typedef struct {
 /* Human-readable text of a status; never NULL. */
 VELOX_API const char *velox_status_string(velox_status s);
 
-/* ABI version of this header (major * 100 + minor): 102. */
+/* ABI version of this header (major * 100 + minor): 103. */
 VELOX_API int velox_abi_version(void);
 
 /*
@@ -498,6 +498,26 @@ VELOX_API velox_status velox_multiwarp(const velox_camera *cams, int n_cams,
 /* Bytes of workspace velox_multiwarp needs: 4 S n_tgt H W. */
 VELOX_API velox_status velox_multiwarp_workspace_size(int S, int n_tgt, int H, int W,
                                                       size_t *bytes);
+
+/*
+ * velox_wait_selftest -- drive the library's bounded waits to their limit.
+ *
+ * The pages have no counterpart: this is the library's failure-detection
+ * check.  Every kernel that waits on an mbarrier bounds the wait by the
+ * device clock; a wait that gives up sets a CTA-wide abort flag, which ends
+ * the CTA's other waits too, and the error is reported through dev_status
+ * instead of a trap.  This call runs that code on one CTA of two warps:
+ * thread 0 waits on a barrier that nothing completes, with a limit of
+ * limit_us microseconds; the 32 threads of the second warp wait on another
+ * such barrier with a limit ten times longer, which only the abort flag can
+ * end at about limit_us.  Each warp that gives up OR-s VELOX_DEV_WAIT_TIMEOUT
+ * into *dev_status.  elapsed_ns (device, nullable) [2] int64: how long thread
+ * 0 and the second warp waited, in ns.  Nothing faults or traps and the
+ * context stays usable.  1 <= limit_us <= 2,000,000, else
+ * VELOX_ERR_INVALID_ARG.
+ */
+VELOX_API velox_status velox_wait_selftest(int limit_us, int32_t *dev_status,
+                                           int64_t *elapsed_ns, velox_stream_t stream);
 
 #ifdef __cplusplus
 }

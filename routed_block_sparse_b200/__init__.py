@@ -43,7 +43,8 @@ EXPORTS = ("velox_status_string", "velox_abi_version", "velox_gilbert_order",
            "velox_block_sparse_attn", "velox_block_importance_noalloc",
            "velox_route_schedule", "velox_two_phase_attn", "velox_slab_overlap",
            "velox_coverage", "velox_route_audit", "velox_thw_linear_order",
-           "velox_slab_table", "velox_multiwarp", "velox_multiwarp_workspace_size")
+           "velox_slab_table", "velox_multiwarp", "velox_multiwarp_workspace_size",
+           "velox_wait_selftest")
 
 
 class VeloxError(RuntimeError):
@@ -104,6 +105,8 @@ def _load() -> ctypes.CDLL:
     lib.velox_two_phase_attn.restype = I
     lib.velox_two_phase_attn.argtypes = [P, P, P, P, P, P, I, P, P, I, I, I, I, I, I, F, P, P, P,
                                          P]
+    lib.velox_wait_selftest.restype = I
+    lib.velox_wait_selftest.argtypes = [I, P, P, P]
     return lib
 
 
@@ -267,3 +270,9 @@ def velox_multiwarp(cams, n_cams, src_depth, src_cam, S, tgt_cam, n_tgt, H, W, s
                               _ptr(tgt_cam), n_tgt, H, W, s, k_warp, _ptr(zq), _ptr(ws),
                               ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream))
     _check("velox_multiwarp", st)
+
+
+def velox_wait_selftest(limit_us, dev_status, elapsed_ns=None, stream=None):
+    st = _lib.velox_wait_selftest(int(limit_us), _ptr(dev_status), _ptr(elapsed_ns),
+                                  _stream(stream))
+    _check("velox_wait_selftest", st)

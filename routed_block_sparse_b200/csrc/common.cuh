@@ -60,19 +60,21 @@ VELOX_DEVFN uint64_t global_timer_ns() {
 }
 
 // Bounded wait for the phase of `parity` to complete.  Gives up after
-// `limit_ns` nanoseconds or as soon as *abort is non-zero; on giving up it
-// sets *abort (so that every other waiter of the CTA stops promptly) and
-// returns false.  Normal runs never come close to the limit.
+// `limit_ns` nanoseconds (2 s unless the caller says otherwise) or as soon as
+// *abort is non-zero; on giving up it sets *abort (so that every other waiter
+// of the CTA stops promptly) and returns false.  Normal runs never come close
+// to the limit.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
-VELOX_DEVFN bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+VELOX_DEVFN bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                           uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort = 1;
         return false;
       }

@@ -60,7 +60,7 @@ def test_binding_names_match_header(built):
 
 def test_status_strings_and_version(built):
     import routed_block_sparse_b200 as rbs
-    assert rbs.velox_abi_version() == 102
+    assert rbs.velox_abi_version() == 103
     for s in range(8):
         assert isinstance(rbs.velox_status_string(s), str) and rbs.velox_status_string(s)
     assert rbs.velox_status_string(99) == "unknown status"
@@ -142,3 +142,15 @@ def test_no_device_is_refused_not_emulated(built):
     # valid arguments, but no sm_100 device: VELOX_ERR_DEVICE (5), nothing runs
     assert lib.velox_gilbert_order(2, 2, 4, 2, 2, 0, 0, 0, fake, None, None, None, None, 0,
                                    None, None) == 5
+    # the wait self-test: valid arguments are refused the same way
+    lib.velox_wait_selftest.restype = ctypes.c_int
+    assert lib.velox_wait_selftest(1000, fake, None, None) == 5
+
+
+def test_wait_selftest_arguments_checked_on_the_host(built):
+    lib = ctypes.CDLL(built)
+    lib.velox_wait_selftest.restype = ctypes.c_int
+    fake = ctypes.c_void_p(0x10000)
+    assert lib.velox_wait_selftest(1000, None, None, None) == 1
+    for bad in (0, -1, 2_000_001):
+        assert lib.velox_wait_selftest(bad, fake, None, None) == 1
