@@ -20,8 +20,12 @@
  * own tiles under one softmax), velox_slab_overlap and velox_coverage (the
  * geometric inputs g and the coverage flags), velox_route_audit (the
  * geometry-model consistency counts), velox_thw_linear_order (the raster
- * order the pages compare the Gilbert order with), velox_route_schedule
- * (longest-route-first row order) and velox_block_importance_noalloc.
+ * order the pages compare the Gilbert order with), velox_slab_table and
+ * velox_multiwarp (the history-side geometry: frustum slabs from depth maps,
+ * the recency-priority multiwarp depth of the current frames),
+ * velox_route_schedule (longest-route-first row order),
+ * velox_block_importance_noalloc and velox_wait_selftest (the bounded waits
+ * driven to their limit).
  *
  * Conventions shared by every call
  * --------------------------------
