@@ -344,7 +344,9 @@ def run_velox(args, world, rank, local):
             with open(tpath) as f:
                 tj = json.load(f)
             if tj.get("kernel_source_hash") == _attn_source_hash():
-                traffic = tj.get("bytes_per_launch")
+                # recorded for a launch of tj["heads"] heads; every head has
+                # the same route statistics and its own K/V
+                traffic = tj["bytes_per_launch"] * wl.heads / tj.get("heads", wl.heads)
         except Exception:
             traffic = None
 
