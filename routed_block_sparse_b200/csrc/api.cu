@@ -128,7 +128,7 @@ velox_status order_common(int T, int H, int W, int n_chunks, int b_tok, int q_ch
                           int32_t *nbr_cnt, int S_max, int thw, int32_t *dev_status,
                           velox_stream_t stream) {
   if (T <= 0 || H <= 0 || W <= 0 || n_chunks <= 0 || b_tok <= 0) return VELOX_ERR_INVALID_ARG;
-  if ((long long)n_chunks * T * H * W > kInt32Max) return VELOX_ERR_UNSUPPORTED;
+  if (velox::product_exceeds({n_chunks, T, H, W}, kInt32Max)) return VELOX_ERR_UNSUPPORTED;
   if (!thw && (W < H || (W % 2 == 1 && H % 2 == 0))) return VELOX_ERR_UNSUPPORTED;
   if (((long long)T * H * W) % b_tok != 0) return VELOX_ERR_UNSUPPORTED;
   if (b_tok > 1024) return VELOX_ERR_UNSUPPORTED;
@@ -188,8 +188,8 @@ velox_status velox_block_importance(const velox_bf16 *Q, const velox_bf16 *K, in
                                     size_t ws_bytes, velox_stream_t stream) {
   if (!Q || !K || !p || H <= 0 || N <= 0 || M <= 0) return VELOX_ERR_INVALID_ARG;
   if (d != VELOX_HEAD_DIM || b_tok != VELOX_BLOCK_TOK) return VELOX_ERR_UNSUPPORTED;
-  if (M > VELOX_MAX_BLOCKS || (long long)H * M * b_tok > kInt32Max ||
-      (long long)H * N * b_tok > kInt32Max)
+  if (M > VELOX_MAX_BLOCKS || velox::product_exceeds({H, M, b_tok}, kInt32Max) ||
+      velox::product_exceeds({H, N, b_tok}, kInt32Max))
     return VELOX_ERR_UNSUPPORTED;
   if (!std::isfinite(scale)) return VELOX_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(p)) return VELOX_ERR_INVALID_ARG;
@@ -375,8 +375,9 @@ velox_status velox_slab_table(const float *depth, const float *conf, const uint8
     return VELOX_ERR_INVALID_ARG;
   if ((long long)(first_block + (long long)n_blocks) * b_tok > n_cells) return VELOX_ERR_INVALID_ARG;
   if (((long long)H * W) % b_tok != 0) return VELOX_ERR_UNSUPPORTED;
-  if ((long long)b_tok * s * s > velox::slab_table_max_samples()) return VELOX_ERR_UNSUPPORTED;
-  if ((long long)F * H * W * s * s > kInt32Max || n_blocks > kInt32Max / 2)
+  if (velox::product_exceeds({b_tok, s, s}, velox::slab_table_max_samples()))
+    return VELOX_ERR_UNSUPPORTED;
+  if (velox::product_exceeds({F, H, W, s, s}, kInt32Max) || n_blocks > kInt32Max / 2)
     return VELOX_ERR_UNSUPPORTED;
   velox_status st = check_device();
   if (st != VELOX_OK) return st;
@@ -400,8 +401,9 @@ velox_status velox_multiwarp(const velox_camera *cams, int n_cams, const float *
     return VELOX_ERR_INVALID_ARG;
   if (n_cams <= 0 || S <= 0 || n_tgt <= 0 || H <= 0 || W <= 0 || s <= 0 || k_warp < 1)
     return VELOX_ERR_INVALID_ARG;
-  if ((long long)H * W * s * s > velox::multiwarp_max_samples() ||
-      (long long)H * W > velox::multiwarp_max_tokens() || n_tgt > 65535 || S > 65535)
+  if (velox::product_exceeds({H, W, s, s}, velox::multiwarp_max_samples()) ||
+      velox::product_exceeds({H, W}, velox::multiwarp_max_tokens()) || n_tgt > 65535 ||
+      S > 65535)
     return VELOX_ERR_UNSUPPORTED;
   if (!ws || ws_bytes < velox::multiwarp_ws_bytes(S, n_tgt, H, W)) return VELOX_ERR_WORKSPACE;
   velox_status st = check_device();

@@ -6,6 +6,7 @@
 #pragma once
 
 #include <cstdint>
+#include <initializer_list>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -14,6 +15,24 @@
 #define VELOX_DEVFN __device__ __forceinline__
 
 namespace velox {
+
+// ----------------------------------------------------- host size checks ---
+// True when the product of the factors exceeds `limit` (or a factor is
+// negative), decided without forming a product that could overflow.
+inline bool product_exceeds(std::initializer_list<long long> factors, long long limit) {
+  bool zero = false;
+  for (long long f : factors) {
+    if (f < 0) return true;
+    if (f == 0) zero = true;
+  }
+  if (zero) return limit < 0;
+  long long prod = 1;
+  for (long long f : factors) {
+    if (prod > limit / f) return true;
+    prod *= f;
+  }
+  return false;
+}
 
 // ---------------------------------------------------------------- status ---
 VELOX_DEVFN void flag_error(int32_t *dev_status, int32_t bits) {

@@ -72,8 +72,8 @@ extern "C" velox_status velox_block_importance_noalloc(const velox_bf16 *Q, cons
                                                        velox_stream_t stream) {
   if (!Q || !K || !p || H <= 0 || N <= 0 || M <= 0) return VELOX_ERR_INVALID_ARG;
   if (d != VELOX_HEAD_DIM || b_tok != VELOX_BLOCK_TOK) return VELOX_ERR_UNSUPPORTED;
-  if (M > VELOX_MAX_BLOCKS || (long long)H * M * b_tok > 2147483647LL ||
-      (long long)H * N * b_tok > 2147483647LL)
+  if (M > VELOX_MAX_BLOCKS || velox::product_exceeds({H, M, b_tok}, 2147483647LL) ||
+      velox::product_exceeds({H, N, b_tok}, 2147483647LL))
     return VELOX_ERR_UNSUPPORTED;
   if (!(scale == scale) || scale - scale != 0.0f) return VELOX_ERR_INVALID_ARG;  // NaN / inf
   if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K) |
