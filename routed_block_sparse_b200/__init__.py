@@ -2,7 +2,10 @@
 
 Argument marshalling only: every function forwards device pointers, sizes
 and the current CUDA stream to the C entry point of the same name declared in
-include/velox.h, and raises VeloxError on a non-OK status.  All compute runs
+include/velox.h, and raises VeloxError on a non-OK status.  Before the call it
+checks what the C ABI cannot see on a raw pointer (each tensor on a CUDA
+device, of the expected dtype, contiguous, with at least the elements the
+sizes imply) and raises ValueError or TypeError otherwise.  All compute runs
 in the library's sm_100a kernels.  Importing this package loads the library
 and raises if it is missing; there is no other implementation to fall back to.
 """
