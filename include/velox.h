@@ -398,8 +398,8 @@ VELOX_API velox_status velox_slab_overlap(const velox_camera *cams, int n_cams,
  * lands in the slab's rectangle at a depth in [zlo, zhi].  z <= 0 (a hole) is
  * never covered.
  *
- * q_uvz [N][b][3] fp32 (u, v, z per token), 1 <= b <= 128; rho [N] fp32,
- * covered [N] uint8 out.
+ * q_uvz [N][b][3] fp32 (u, v, z per token), 1 <= b <= 128, N <= 2^29 (four
+ * CTAs per query block); rho [N] fp32, covered [N] uint8 out.
  */
 VELOX_API velox_status velox_coverage(const velox_camera *cams, int n_cams,
                                       const velox_slab *q_slabs, const float *q_uvz, int N,

@@ -338,7 +338,7 @@ velox_status velox_coverage(const velox_camera *cams, int n_cams, const velox_sl
   if (!cams || !q_slabs || !q_uvz || !h_slabs || !rho || !covered || !dev_status)
     return VELOX_ERR_INVALID_ARG;
   if (n_cams <= 0 || N <= 0 || M <= 0 || b <= 0 || std::isnan(eta)) return VELOX_ERR_INVALID_ARG;
-  if (b > 128) return VELOX_ERR_UNSUPPORTED;
+  if (b > 128 || N > kInt32Max / 4) return VELOX_ERR_UNSUPPORTED;  // 4 CTAs per query block
   velox_status st = check_device();
   if (st != VELOX_OK) return st;
   return from_cuda(velox::launch_coverage(cams, n_cams, q_slabs, q_uvz, N, b, h_slabs, M, eta, rho,

@@ -123,3 +123,64 @@ def test_the_overflowing_products_are_refused(lib):
                                 0.1, 0.9, FAKE, None, FAKE, None) == 2
     assert lib.velox_multiwarp(FAKE, 4, FAKE, FAKE, 1, FAKE, 1, 2**16, 2**16, 2**16, 2, FAKE,
                                FAKE, 2**62, FAKE, None) == 2
+
+
+class _Prm(ctypes.Structure):
+    _fields_ = [("lam", ctypes.c_float), ("tau", ctypes.c_float), ("g_ref", ctypes.c_float),
+                ("theta_cov", ctypes.c_float), ("theta_unc", ctypes.c_float),
+                ("k_cov", ctypes.c_int32), ("k_unc", ctypes.c_int32)]
+
+
+@settings(max_examples=400, deadline=None)
+@given(H=sizes, N=sizes, M=sizes, R_max=sizes, k_cov=sizes, k_unc=sizes, prev_begin=sizes,
+       prev_count=sizes, S_max=sizes)
+def test_route_build_sizes(lib, H, N, M, R_max, k_cov, k_unc, prev_begin, prev_count, S_max):
+    f = lib.velox_route_build
+    f.restype = ctypes.c_int
+    prm = _Prm(2.0, 0.1, 0.2, 0.9, 0.9, k_cov, k_unc)
+    nbr = FAKE if S_max > 0 else None
+    s = f(FAKE, FAKE, FAKE, ctypes.byref(prm), prev_begin, prev_count, nbr, nbr, S_max, None, 0,
+          H, N, M, FAKE, FAKE, FAKE, R_max, FAKE, ctypes.c_size_t(2**62), FAKE, None)
+    assert s in STATUSES
+    if s == OK_DEVICE:
+        assert min(H, N, M) > 0 and M <= 65536 and H * N <= I32 // 2
+        assert 0 <= prev_begin and 0 <= prev_count and prev_begin + prev_count <= M
+        assert 0 <= k_cov <= 4096 and 0 <= k_unc <= 4096 and S_max >= 0
+        assert R_max >= min(M, max(k_cov, k_unc, prev_count) + max(S_max, 0)) and R_max > 0
+
+
+@settings(max_examples=300, deadline=None)
+@given(N=sizes, M=sizes, grid=sizes, n_cams=sizes, b=sizes)
+def test_geometry_sizes(lib, N, M, grid, n_cams, b):
+    f = lib.velox_slab_overlap
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                  ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    s = f(FAKE, n_cams, FAKE, N, FAKE, M, grid, FAKE, FAKE, None)
+    assert s in STATUSES
+    if s == OK_DEVICE:
+        assert min(N, M, grid, n_cams) > 0 and grid <= 32 and N <= 65535 and N * M <= I32
+    c = lib.velox_coverage
+    c.restype = ctypes.c_int
+    c.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                  ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    s = c(FAKE, n_cams, FAKE, FAKE, N, b, FAKE, M, 0.9, FAKE, FAKE, FAKE, None)
+    assert s in STATUSES
+    if s == OK_DEVICE:
+        assert min(N, M, b, n_cams) > 0 and b <= 128 and 4 * N <= I32
+
+
+@settings(max_examples=300, deadline=None)
+@given(H=sizes, N=sizes, M=sizes, k_geo=sizes, k_fuse=sizes)
+def test_audit_sizes(lib, H, N, M, k_geo, k_fuse):
+    f = lib.velox_route_audit
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    prm = _Prm(2.0, 0.1, 0.2, 0.9, 0.9, 80, 150)
+    s = f(FAKE, FAKE, H, N, M, ctypes.byref(prm), k_geo, k_fuse, FAKE, None)
+    assert s in STATUSES
+    if s == OK_DEVICE:
+        assert min(H, N, M) > 0 and k_geo >= 1 and k_fuse >= 1
+        assert M <= 4096 and H * N <= I32
