@@ -24,6 +24,13 @@ adjacent where a literal per-chunk mirror would break them.  Halving in the
 curve construction rounds toward minus infinity (floor division).  Supported
 frames have W >= H and are not (W odd, H even), the case in which no unit-step
 path from (0, 0) to (W-1, 0) exists.
+
+Pins (tests/test_oracle_gilbert.py): a bijection with unit steps across every
+block, frame and chunk seam; contiguous chunks; the mirror rule; and, on
+2^k x 2^k frames, the textbook Hilbert curve cell for cell.  On other frame
+shapes (the 32 x 48 latent frame among them), which unit-step path the
+construction picks is fixed only by those invariants.  Against the authors'
+own figures it is parity unpinned: the figures' ranks are not in the text.
 """
 
 from __future__ import annotations
