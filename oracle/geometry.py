@@ -31,128 +31,222 @@ Readings taken where the pages are open:
   r's camera, lands in the rectangle [u0, u1) x [v0, v1) at a depth in
   [z-, z+]; a token with depth <= 0 (a hole) is never covered.
 
-The inside/outside decisions turn floats into counts, so they are taken in
-fp32 with the same operation order as the CUDA kernel (every product and sum
-rounded separately, in the order written here); the ratios are fp64.
+Everything here is plain fp64 arithmetic from the fp32 inputs (numpy matrix
+products, no imposed operation order).  The inside/outside decisions turn
+floats into counts, and an implementation in another precision may decide a
+point that lies within rounding distance of a face the other way.  So every
+decision also yields its distance to the deciding face, in world units; a
+decision closer than EPS_REL x (the size of the coordinates involved) is
+"marginal".  The *_bounds functions return, next to the value, the values
+that every choice of the marginal decisions can give: a count in
+[n_lo, n_hi] and the matching g or rho interval.
 """
 
 from __future__ import annotations
 
 import numpy as np
 
-F = np.float32
+# Relative size of a marginal decision.  An fp32 evaluation of these
+# formulas (about 20 roundings of coordinates of size s) lands within a few
+# 1e-6 s of the fp64 value; 1e-5 s leaves a margin of several times that.
+EPS_REL = 1e-5
 
 
-def _f(x):
-    return np.asarray(x, dtype=np.float32)
+def _cam(cam):
+    c = np.asarray(cam, dtype=np.float64)
+    return c[0], c[1], c[2], c[3], c[4:13].reshape(3, 3), c[13:16]
 
 
 def obb(cam: np.ndarray, slab: np.ndarray):
-    """Centre (3,), axes R (3x3, columns) and half extents (3,) of a slab.
+    """Centre (3,), axes R (3x3, columns) and half extents (3,) of a slab, fp64.
 
     cam: [fx, fy, cx, cy, R00..R22 (row-major), Cx, Cy, Cz] (16 fp32)
     slab: [u0, u1, v0, v1, zlo, zhi] (fp32)
     """
-    cam, slab = _f(cam), _f(slab)
-    fx, fy, cx, cy = cam[0], cam[1], cam[2], cam[3]
-    R = cam[4:13].reshape(3, 3)
-    C = cam[13:16]
-    u0, u1, v0, v1, zlo, zhi = slab[:6]
-    zm = F(0.5) * F(zlo + zhi)
-    um = F(0.5) * F(u0 + u1)
-    vm = F(0.5) * F(v0 + v1)
-    xl = F(F(F(um - cx) / fx) * zm)
-    yl = F(F(F(vm - cy) / fy) * zm)
-    centre = _cam_to_world(R, C, np.array([xl, yl, zm], dtype=F))
-    half = np.array([F(F(F(F(u1 - u0) * F(0.5)) / fx) * zm),
-                     F(F(F(F(v1 - v0) * F(0.5)) / fy) * zm),
-                     F(F(0.5) * F(zhi - zlo))], dtype=F)
+    fx, fy, cx, cy, R, C = _cam(cam)
+    u0, u1, v0, v1, zlo, zhi = np.asarray(slab, dtype=np.float64)[:6]
+    zm = 0.5 * (zlo + zhi)
+    local = np.array([(0.5 * (u0 + u1) - cx) / fx * zm, (0.5 * (v0 + v1) - cy) / fy * zm, zm])
+    centre = C + R @ local
+    half = np.array([(u1 - u0) / (2.0 * fx) * zm, (v1 - v0) / (2.0 * fy) * zm,
+                     0.5 * (zhi - zlo)])
     return centre, R, half
 
 
-def _cam_to_world(R, C, x):
-    """C + R x with the kernel's rounding order: ((R0 x0 + R1 x1) + R2 x2) + C."""
-    out = np.empty(3, dtype=F)
-    for k in range(3):
-        acc = F(R[k, 0] * x[0])
-        acc = F(acc + F(R[k, 1] * x[1]))
-        acc = F(acc + F(R[k, 2] * x[2]))
-        out[k] = F(acc + C[k])
-    return out
+def _grid_points(ci, Ri, hi, G):
+    """World positions of the G^3 cell centres of a box: [G^3][3] (a, b, c order)."""
+    s = (2.0 * np.arange(G) + 1.0) / G - 1.0
+    a, b, c = np.meshgrid(s, s, s, indexing="ij")
+    local = np.stack([a.ravel() * hi[0], b.ravel() * hi[1], c.ravel() * hi[2]], axis=1)
+    return ci + local @ Ri.T
 
 
-def _world_to_box(R, centre, X):
-    """R^T (X - centre), same rounding order."""
-    dx = np.array([F(X[0] - centre[0]), F(X[1] - centre[1]), F(X[2] - centre[2])], dtype=F)
-    out = np.empty(3, dtype=F)
-    for k in range(3):
-        acc = F(R[0, k] * dx[0])
-        acc = F(acc + F(R[1, k] * dx[1]))
-        acc = F(acc + F(R[2, k] * dx[2]))
-        out[k] = acc
-    return out
+def slab_iou_counts(cam_i, slab_i, cam_r, slab_r, valid_r: bool, grid: int):
+    """(n_in, n_lo, n_hi, vol_i, vol_r) of one (query, history) slab pair.
 
-
-def slab_iou(cam_i, slab_i, cam_r, slab_r, valid_r: bool, grid: int) -> float:
-    """g for one (query slab, history slab) pair."""
+    n_in counts the query box's grid points inside the history box; n_lo
+    those inside by more than the marginal distance, n_hi those inside or
+    outside by less than it.  An invalid history slab gives all zeros.
+    """
+    G = grid
     if not valid_r:
-        return 0.0
+        return 0, 0, 0, 0.0, 0.0
     ci, Ri, hi = obb(cam_i, slab_i)
     cr, Rr, hr = obb(cam_r, slab_r)
-    G = grid
-    s = [F(F(F(2 * a + 1) / F(G)) - F(1.0)) for a in range(G)]
-    n_in = 0
-    for a in range(G):
-        for b in range(G):
-            for c in range(G):
-                p = np.array([F(s[a] * hi[0]), F(s[b] * hi[1]), F(s[c] * hi[2])], dtype=F)
-                X = _cam_to_world(Ri, ci, p)
-                d = _world_to_box(Rr, cr, X)
-                if abs(d[0]) <= hr[0] and abs(d[1]) <= hr[1] and abs(d[2]) <= hr[2]:
-                    n_in += 1
-    vi = 8.0 * float(hi[0]) * float(hi[1]) * float(hi[2])
-    vr = 8.0 * float(hr[0]) * float(hr[1]) * float(hr[2])
-    inter = vi * n_in / float(G ** 3)
+    X = _grid_points(ci, Ri, hi, G)
+    d = (X - cr) @ Rr                      # box-frame coordinates R_r^T (X - c_r)
+    margin = np.min(hr[None, :] - np.abs(d), axis=1)   # > 0 inside, < 0 outside
+    scale = max(1.0, float(np.abs(X).max()), float(np.abs(cr).max()), float(hr.max()))
+    eps = EPS_REL * scale
+    n_in = int(np.count_nonzero(margin >= 0.0))
+    n_lo = int(np.count_nonzero(margin > eps))
+    n_hi = int(np.count_nonzero(margin >= -eps))
+    vi = 8.0 * hi[0] * hi[1] * hi[2]
+    vr = 8.0 * hr[0] * hr[1] * hr[2]
+    return n_in, n_lo, n_hi, vi, vr
+
+
+def iou_from_count(n: int, vi: float, vr: float, grid: int) -> float:
+    """IoU for an inside count n: inter = vi n / G^3, g = inter / (vi + vr - inter)."""
+    inter = vi * n / float(grid ** 3)
     union = vi + vr - inter
     return inter / union if union > 0.0 else 0.0
 
 
-def overlap(cams, q_cam, q_slab, h_cam, h_slab, h_valid, grid: int) -> np.ndarray:
-    """g [N][M] for all query slabs against all history slabs."""
+def slab_iou(cam_i, slab_i, cam_r, slab_r, valid_r: bool, grid: int) -> float:
+    """g for one (query slab, history slab) pair."""
+    n, _, _, vi, vr = slab_iou_counts(cam_i, slab_i, cam_r, slab_r, valid_r, grid)
+    return iou_from_count(n, vi, vr, grid) if valid_r else 0.0
+
+
+def overlap_bounds(cams, q_cam, q_slab, h_cam, h_slab, h_valid, grid: int):
+    """g, g_lo, g_hi [N][M]: the IoU and its range over the marginal decisions."""
     N, M = len(q_cam), len(h_cam)
     g = np.zeros((N, M))
+    lo = np.zeros((N, M))
+    hi = np.zeros((N, M))
     for i in range(N):
         for r in range(M):
-            g[i, r] = slab_iou(cams[q_cam[i]], q_slab[i], cams[h_cam[r]], h_slab[r],
-                               bool(h_valid[r]), grid)
-    return g
+            n, n_lo, n_hi, vi, vr = slab_iou_counts(cams[q_cam[i]], q_slab[i], cams[h_cam[r]],
+                                                    h_slab[r], bool(h_valid[r]), grid)
+            if h_valid[r]:
+                g[i, r] = iou_from_count(n, vi, vr, grid)
+                lo[i, r] = iou_from_count(n_lo, vi, vr, grid)
+                hi[i, r] = iou_from_count(n_hi, vi, vr, grid)
+    return g, lo, hi
 
 
-def _project(cam, X):
-    """(u, v, z) of world point X in camera `cam`, kernel rounding order."""
-    cam = _f(cam)
-    fx, fy, cx, cy = cam[0], cam[1], cam[2], cam[3]
-    R = cam[4:13].reshape(3, 3)
-    x = _world_to_box(R, cam[13:16], X)  # camera frame: R^T (X - C)
-    z = x[2]
-    u = F(F(F(x[0] / z) * fx) + cx)
-    v = F(F(F(x[1] / z) * fy) + cy)
-    return u, v, z
+def overlap(cams, q_cam, q_slab, h_cam, h_slab, h_valid, grid: int) -> np.ndarray:
+    """g [N][M] for all query slabs against all history slabs."""
+    return overlap_bounds(cams, q_cam, q_slab, h_cam, h_slab, h_valid, grid)[0]
+
+
+def token_world(cam_t, u, v, z) -> np.ndarray:
+    """World point of token (u, v) at depth z of camera cam_t."""
+    fx, fy, cx, cy, R, C = _cam(cam_t)
+    u, v, z = float(u), float(v), float(z)
+    return C + R @ np.array([(u - cx) / fx * z, (v - cy) / fy * z, z])
+
+
+def inside_margin(X: np.ndarray, cam_r, slab_r):
+    """(inside, margin) of world point X against slab r: inside when X
+    projects into [u0, u1) x [v0, v1) at a depth in [z-, z+]; margin is the
+    distance to the nearest face of that frustum piece in world units
+    (image-plane distances times depth / focal length), as a lower bound of
+    how far X can move before the decision changes."""
+    fx, fy, cx, cy, R, C = _cam(cam_r)
+    d = R.T @ (X - C)
+    pz = d[2]
+    if pz <= 0.0:
+        return False, float(-pz)
+    pu = d[0] / pz * fx + cx
+    pv = d[1] / pz * fy + cy
+    u0, u1, v0, v1, zlo, zhi = np.asarray(slab_r, dtype=np.float64)[:6]
+    inside = (u0 <= pu < u1) and (v0 <= pv < v1) and (zlo <= pz <= zhi)
+    du = min(abs(pu - u0), abs(u1 - pu)) * pz / fx
+    dv = min(abs(pv - v0), abs(v1 - pv)) * pz / fy
+    dz = min(abs(pz - zlo), abs(zhi - pz))
+    if inside:
+        margin = min(du, dv, dz)
+    else:
+        # outside: the distance to the nearest violated face bounds the move
+        # needed to become inside from below by that face alone
+        viol = []
+        if not (u0 <= pu < u1):
+            viol.append(du)
+        if not (v0 <= pv < v1):
+            viol.append(dv)
+        if not (zlo <= pz <= zhi):
+            viol.append(dz)
+        margin = max(viol)
+    return bool(inside), float(margin)
 
 
 def token_inside(cam_t, u, v, z, cam_r, slab_r) -> bool:
     """Does token (u, v) at depth z of camera cam_t fall inside slab r?"""
     if not z > 0:
         return False
-    cam_t = _f(cam_t)
-    fx, fy, cx, cy = cam_t[0], cam_t[1], cam_t[2], cam_t[3]
-    R = cam_t[4:13].reshape(3, 3)
-    xl = F(F(F(F(u) - cx) / fx) * F(z))
-    yl = F(F(F(F(v) - cy) / fy) * F(z))
-    X = _cam_to_world(R, cam_t[13:16], np.array([xl, yl, F(z)], dtype=F))
-    pu, pv, pz = _project(cam_r, X)
-    s = _f(slab_r)
-    return bool(pz > 0 and s[0] <= pu < s[1] and s[2] <= pv < s[3] and s[4] <= pz <= s[5])
+    return inside_margin(token_world(cam_t, u, v, z), cam_r, slab_r)[0]
+
+
+def _inside_margin_many(X: np.ndarray, cams_r: np.ndarray, slabs_r: np.ndarray):
+    """inside_margin of one world point against many slabs at once: the same
+    formulas, one row per slab (cams_r [n][16], slabs_r [n][6])."""
+    c = np.asarray(cams_r, dtype=np.float64)
+    fx, fy, cx, cy = c[:, 0], c[:, 1], c[:, 2], c[:, 3]
+    R = c[:, 4:13].reshape(-1, 3, 3)
+    C = c[:, 13:16]
+    d = np.einsum("nji,nj->ni", R, X[None, :] - C)   # R^T (X - C) per slab
+    pz = d[:, 2]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        pu = d[:, 0] / pz * fx + cx
+        pv = d[:, 1] / pz * fy + cy
+    sl = np.asarray(slabs_r, dtype=np.float64)
+    u0, u1, v0, v1, zlo, zhi = (sl[:, k] for k in range(6))
+    in_u = (u0 <= pu) & (pu < u1)
+    in_v = (v0 <= pv) & (pv < v1)
+    in_z = (zlo <= pz) & (pz <= zhi)
+    front = pz > 0.0
+    inside = front & in_u & in_v & in_z
+    du = np.minimum(np.abs(pu - u0), np.abs(u1 - pu)) * pz / fx
+    dv = np.minimum(np.abs(pv - v0), np.abs(v1 - pv)) * pz / fy
+    dz = np.minimum(np.abs(pz - zlo), np.abs(zhi - pz))
+    m_in = np.minimum(np.minimum(du, dv), dz)
+    m_out = np.maximum(np.maximum(np.where(in_u, 0.0, du), np.where(in_v, 0.0, dv)),
+                       np.where(in_z, 0.0, dz))
+    margin = np.where(front, np.where(inside, m_in, m_out), -pz)
+    return inside, margin
+
+
+def coverage_bounds(cams, q_cam, q_uvz, h_cam, h_slab, h_valid):
+    """Covered token counts n, n_lo, n_hi [N] of every query block.
+
+    A token counts in n when some valid slab holds it; in n_lo when some
+    valid slab holds it by more than the marginal distance; in n_hi when some
+    valid slab holds it or misses it by less than the marginal distance.
+    """
+    N, b = q_uvz.shape[0], q_uvz.shape[1]
+    n = np.zeros(N, dtype=np.int64)
+    n_lo = np.zeros(N, dtype=np.int64)
+    n_hi = np.zeros(N, dtype=np.int64)
+    valid = np.flatnonzero(np.asarray(h_valid) != 0)
+    cams = np.asarray(cams)
+    cams_r = cams[np.asarray(h_cam)[valid]]
+    slabs_r = np.asarray(h_slab)[valid]
+    c_size = np.abs(cams_r[:, 13:16].astype(np.float64)).max(axis=1) if len(valid) else None
+    for i in range(N):
+        cam_t = cams[q_cam[i]]
+        for t in range(b):
+            u, v, z = (float(x) for x in q_uvz[i, t])
+            if not z > 0 or len(valid) == 0:
+                continue  # a hole is never covered
+            X = token_world(cam_t, u, v, z)
+            eps = EPS_REL * np.maximum(max(1.0, float(np.abs(X).max())), c_size)
+            inside, margin = _inside_margin_many(X, cams_r, slabs_r)
+            n[i] += bool(inside.any())
+            n_lo[i] += bool((inside & (margin > eps)).any())
+            n_hi[i] += bool((inside | (margin <= eps)).any())
+    return n, n_lo, n_hi
 
 
 def coverage(cams, q_cam, q_uvz, h_cam, h_slab, h_valid, eta: float = 0.9):
@@ -160,15 +254,7 @@ def coverage(cams, q_cam, q_uvz, h_cam, h_slab, h_valid, eta: float = 0.9):
 
     q_uvz: [N][b][3] token coordinates and warped depth of each query block.
     """
-    N, b = q_uvz.shape[0], q_uvz.shape[1]
-    rho = np.zeros(N)
-    for i in range(N):
-        n_cov = 0
-        for t in range(b):
-            u, v, z = q_uvz[i, t]
-            for r in range(len(h_cam)):
-                if h_valid[r] and token_inside(cams[q_cam[i]], u, v, z, cams[h_cam[r]], h_slab[r]):
-                    n_cov += 1
-                    break
-        rho[i] = n_cov / b
+    b = q_uvz.shape[1]
+    n, _, _ = coverage_bounds(cams, q_cam, q_uvz, h_cam, h_slab, h_valid)
+    rho = n / b
     return rho, (rho >= float(np.float32(eta))).astype(np.uint8)

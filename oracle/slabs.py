@@ -36,10 +36,13 @@ Readings taken where the pages are open:
   hole (depth 0);
 * blocks never straddle frames (H W is a multiple of the block size).
 
-The projections use the fp32 operation order of ``oracle.geometry`` (every
-product, sum and quotient rounded separately): the target token of a sample
-is an integer decided by floats, so both sides decide it in fp32 the same
-way.
+The projections are plain fp64 arithmetic from the fp32 inputs (the
+formulas of ``oracle.geometry``).  The target token of a sample is an integer
+decided by floats: a sample whose projected position lies within the
+marginal distance of a token edge (EPS_REL of ``oracle.geometry``, in world
+units) could land in either neighbour in another precision, so the multiwarp
+also reports the target tokens that such a sample touches ("unsure" tokens,
+whose count, source and median are not fixed by the fp64 decision).
 """
 
 from __future__ import annotations
@@ -50,7 +53,7 @@ from typing import List, Sequence
 
 import numpy as np
 
-from .geometry import _cam_to_world, _world_to_box
+from .geometry import EPS_REL, _cam, token_world
 
 F = np.float32
 
@@ -137,43 +140,63 @@ def block_tokens(depth, conf, mask, cell_of_rank, H: int, W: int, b: int, frame_
 
 
 def warp_sample(cam_src, cam_tgt, u, v, z, H: int, W: int):
-    """Target token (x, y) and target depth of source point (u, v) at depth z,
-    or None when it does not land in the target frame."""
-    cs = np.asarray(cam_src, dtype=F)
-    fx, fy, cx, cy = cs[0], cs[1], cs[2], cs[3]
-    xl = F(F(F(F(u) - cx) / fx) * F(z))
-    yl = F(F(F(F(v) - cy) / fy) * F(z))
-    X = _cam_to_world(cs[4:13].reshape(3, 3), cs[13:16], np.array([xl, yl, F(z)], dtype=F))
-    ct = np.asarray(cam_tgt, dtype=F)
-    d = _world_to_box(ct[4:13].reshape(3, 3), ct[13:16], X)
-    if not d[2] > 0:
-        return None
-    pu = F(F(F(d[0] / d[2]) * ct[0]) + ct[2])
-    pv = F(F(F(d[1] / d[2]) * ct[1]) + ct[3])
-    if not (F(0) <= pu < F(W) and F(0) <= pv < F(H)):
-        return None
-    return int(math.floor(pu)), int(math.floor(pv)), float(d[2])
+    """Warp source point (u, v) at depth z into the target camera.
+
+    Returns (cell, depth, margin, candidates): cell = (x, y) of the target
+    token it lands in, or None when it does not land in the frame (target
+    depth <= 0 or outside [0, W) x [0, H)); depth = the target-camera depth;
+    margin = the distance in world units to the nearest token edge (frame
+    edges included) or to the camera plane; candidates = the in-frame cells
+    the point lies in or touches within the marginal distance.
+    """
+    X = token_world(cam_src, u, v, z)
+    fx, fy, cx, cy, R, C = _cam(cam_tgt)
+    d = R.T @ (X - C)
+    pz = float(d[2])
+    eps = EPS_REL * max(1.0, float(np.abs(X).max()), float(np.abs(C).max()))
+    if not pz > 0.0:
+        return None, pz, -pz, []
+    pu = d[0] / pz * fx + cx
+    pv = d[1] / pz * fy + cy
+    mu = abs(pu - round(pu)) * pz / fx
+    mv = abs(pv - round(pv)) * pz / fy
+    margin = min(mu, mv, pz)
+    du, dv = eps * fx / pz, eps * fy / pz          # the marginal distance in token units
+    xs = {math.floor(pu - du), math.floor(pu), math.floor(pu + du)}
+    ys = {math.floor(pv - dv), math.floor(pv), math.floor(pv + dv)}
+    cand = [(x, y) for x in xs for y in ys if 0 <= x < W and 0 <= y < H]
+    if not (0.0 <= pu < W and 0.0 <= pv < H):
+        return None, pz, margin, cand
+    return (math.floor(pu), math.floor(pv)), pz, margin, cand
 
 
-def multiwarp(cams, src_depth, src_cam: Sequence[int], tgt_cam: int, H: int, W: int, s: int,
-              k_warp: int = 2) -> np.ndarray:
+def multiwarp_bounds(cams, src_depth, src_cam: Sequence[int], tgt_cam: int, H: int, W: int,
+                     s: int, k_warp: int = 2):
     """z^Q [H][W] of the target camera from source depths [S][H s][W s]
-    (src_cam[k] is the camera of source k, newest first)."""
+    (src_cam[k] is the camera of source k, newest first), and the [H][W]
+    mask of unsure tokens (touched by a sample whose landing is marginal)."""
     S = len(src_cam)
     per_src: List[dict] = []
+    unsure = np.zeros((H, W), dtype=bool)
     for k in range(S):
         got: dict = {}
         dk = src_depth[k]
+        cam_s, cam_t = cams[src_cam[k]], cams[tgt_cam]
         for py in range(H * s):
             for px in range(W * s):
                 z = float(dk[py, px])
                 if not z > 0.0:
                     continue
-                u = F(F(F(px) + F(0.5)) / F(s))
-                v = F(F(F(py) + F(0.5)) / F(s))
-                hit = warp_sample(cams[src_cam[k]], cams[tgt_cam], u, v, z, H, W)
-                if hit is not None:
-                    got.setdefault((hit[0], hit[1]), []).append(hit[2])
+                u = (px + 0.5) / s
+                v = (py + 0.5) / s
+                cell, depth, margin, cand = warp_sample(cam_s, cam_t, u, v, z, H, W)
+                eps = EPS_REL * max(1.0, float(np.abs(token_world(cam_s, u, v, z)).max()),
+                                    float(np.abs(np.asarray(cam_t, np.float64)[13:16]).max()))
+                if margin <= eps:
+                    for (x, y) in cand:
+                        unsure[y, x] = True
+                if cell is not None:
+                    got.setdefault(cell, []).append(depth)
         per_src.append(got)
     zq = np.zeros((H, W), dtype=np.float32)
     for y in range(H):
@@ -181,11 +204,12 @@ def multiwarp(cams, src_depth, src_cam: Sequence[int], tgt_cam: int, H: int, W: 
             for got in per_src:
                 vals = got.get((x, y), [])
                 if len(vals) >= k_warp:
-                    vals = sorted(vals)
-                    n = len(vals)
-                    if n % 2 == 1:
-                        zq[y, x] = vals[n // 2]
-                    else:
-                        zq[y, x] = F((vals[n // 2 - 1] + vals[n // 2]) / 2.0)
+                    zq[y, x] = np.float32(np.median(np.asarray(vals, dtype=np.float64)))
                     break
-    return zq
+    return zq, unsure
+
+
+def multiwarp(cams, src_depth, src_cam: Sequence[int], tgt_cam: int, H: int, W: int, s: int,
+              k_warp: int = 2) -> np.ndarray:
+    """z^Q [H][W] of the target camera (see multiwarp_bounds)."""
+    return multiwarp_bounds(cams, src_depth, src_cam, tgt_cam, H, W, s, k_warp)[0]

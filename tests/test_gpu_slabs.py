@@ -1,7 +1,15 @@
 """Slab-table build, multiwarp and the whole geometry chain on the GPU vs the
-oracle: rectangles, cameras, flags and token targets exact; percentiles and
-medians bit-exact (both sides take them in fp64 from the fp32 samples and
-round once); g and coverage as in the geometry tests."""
+fp64 oracle.
+
+Slab tables: rectangles, cameras and flags exact, and the percentiles
+bit-exact (both sides interpolate the order statistics of the fp32 samples
+in fp64 and round once to fp32: the reading of "10/90 percentile" fixes the
+precision).  Multiwarp: the landing token of a sample is an integer decided
+by floats; tokens that no marginal sample touches must have the oracle's
+hole pattern and depths within MW_RTOL (tests/parity.py), and the marginal
+ones are counted and bounded.  The chain test checks every stage against
+the oracle applied to that stage's own GPU inputs, so the margins of one
+stage do not leak into the next."""
 
 import numpy as np
 import pytest
@@ -11,7 +19,7 @@ import routed_block_sparse_b200 as rbs
 from oracle import geometry as geo
 from oracle import gilbert
 from oracle import slabs as osl
-from parity import G_RTOL
+from parity import check_coverage_bounds, check_g_bounds, check_multiwarp
 from synth.depth import make_rollout
 from synth.geometry import pack_slabs
 
@@ -111,8 +119,8 @@ def test_multiwarp_matches_oracle(lib, H, W, s, k):
     zq, st = _gpu_multiwarp(r.cams, r.depth[src], src, tgt, H, W, s, k)
     assert st == 0
     for j, t in enumerate(tgt):
-        ref = osl.multiwarp(r.cams, r.depth[src], src, t, H, W, s, k)
-        assert np.array_equal(zq[j], ref)
+        ref, unsure = osl.multiwarp_bounds(r.cams, r.depth[src], src, t, H, W, s, k)
+        check_multiwarp(zq[j], ref, unsure)
     if k <= s * s:  # s x s samples per source token: k_warp above that rarely holds
         assert (zq > 0).mean() > 0.3
 
@@ -122,8 +130,9 @@ def test_multiwarp_chunk48_frame(lib):
     r = make_rollout(4, 192, H, W, s)
     src = [183, 180, 179, 176]
     zq, st = _gpu_multiwarp(r.cams, r.depth[src], src, [188], H, W, s, 2)
-    ref = osl.multiwarp(r.cams, r.depth[src], src, 188, H, W, s, 2)
-    assert st == 0 and np.array_equal(zq[0], ref) and (ref > 0).mean() > 0.9
+    ref, unsure = osl.multiwarp_bounds(r.cams, r.depth[src], src, 188, H, W, s, 2)
+    assert st == 0 and (ref > 0).mean() > 0.9
+    check_multiwarp(zq[0], ref, unsure)
 
 
 def test_multiwarp_bad_camera_is_flagged(lib):
@@ -131,13 +140,14 @@ def test_multiwarp_bad_camera_is_flagged(lib):
     r = make_rollout(1, 4, H, W, s)
     zq, st = _gpu_multiwarp(r.cams, r.depth[[1, 2]], [99, 2], [3], H, W, s, 2)
     assert st & rbs.DEV_BAD_CAMERA
-    ref = osl.multiwarp(r.cams, r.depth[[2]], [2], 3, H, W, s, 2)
-    assert np.array_equal(zq[0], ref)
+    ref, unsure = osl.multiwarp_bounds(r.cams, r.depth[[2]], [2], 3, H, W, s, 2)
+    check_multiwarp(zq[0], ref, unsure)
 
 
 def test_geometry_chain_depth_to_g_and_coverage(lib):
     """Depth maps -> history slab table -> multiwarp query depth -> query slabs
-    and tokens -> slab overlap and coverage, GPU chain against oracle chain."""
+    and tokens -> slab overlap and coverage: every GPU stage against the
+    oracle applied to that stage's GPU inputs."""
     T, H, W, b, nc, s = 4, 8, 16, 32, 6, 2
     q_chunk = nc - 1
     r = make_rollout(11, nc * T, H, W, s, step=0.05)
@@ -152,22 +162,26 @@ def test_geometry_chain_depth_to_g_and_coverage(lib):
     assert st == 0
     ref_h = osl.slab_table(r.depth[:hist_frames], r.conf[:hist_frames], r.mask[:hist_frames], cr,
                            H, W, b, 0, 0, M, prm)
-    assert np.array_equal(hs, ref_h[0]) and np.array_equal(hv, ref_h[2])
+    assert np.array_equal(hs, ref_h[0]) and np.array_equal(hc, ref_h[1])
+    assert np.array_equal(hv, ref_h[2])
     # query depth of the current chunk's frames from the newest history frames
     src = list(range(hist_frames - 1, hist_frames - 9, -1))
     tgt = list(range(hist_frames, hist_frames + T))
     zq, st = _gpu_multiwarp(r.cams, r.depth[src], src, tgt, H, W, s, 2)
     assert st == 0
-    zq_ref = np.stack([osl.multiwarp(r.cams, r.depth[src], src, t, H, W, s, 2) for t in tgt])
-    assert np.array_equal(zq, zq_ref)
+    for j, t in enumerate(tgt):
+        ref, unsure = osl.multiwarp_bounds(r.cams, r.depth[src], src, t, H, W, s, 2)
+        check_multiwarp(zq[j], ref, unsure)
+    # query slabs and tokens from the GPU's multiwarp depth
     qprm = osl.SlabParams(s=1, n_min=8)
     first_q = q_chunk * per_chunk
     qs, qc, qv, st, quvz = _gpu_slabs(zq, None, None, hist_frames, H, W, 1, cell, b, first_q,
                                       per_chunk, qprm, uvz=True)
     assert st == 0
-    ref_q = osl.slab_table(zq_ref, None, None, cr, H, W, b, hist_frames, first_q, per_chunk, qprm)
+    ref_q = osl.slab_table(zq, None, None, cr, H, W, b, hist_frames, first_q, per_chunk, qprm)
     assert np.array_equal(qs, ref_q[0]) and np.array_equal(qc, ref_q[1])
-    ref_uvz = osl.block_tokens(zq_ref, None, None, cr, H, W, b, hist_frames, first_q, per_chunk)
+    assert np.array_equal(qv, ref_q[2])
+    ref_uvz = osl.block_tokens(zq, None, None, cr, H, W, b, hist_frames, first_q, per_chunk)
     assert np.array_equal(quvz, ref_uvz)
     # overlap and coverage on the chain's slabs (query slabs kept valid: the
     # overlap of a query block is defined whatever its own n_min)
@@ -184,11 +198,8 @@ def test_geometry_chain_depth_to_g_and_coverage(lib):
                        0.9, rho, cov, stt)
     torch.cuda.synchronize()
     assert int(stt.item()) == 0
-    g_ref = geo.overlap(r.cams, qc, qs, hc, hs, hv, 8)
-    gg = g.cpu().numpy().astype(np.float64)
-    assert np.array_equal(gg == 0, g_ref == 0) and (g_ref > 0).any()
-    nz = g_ref != 0
-    assert np.all(np.abs(gg[nz] / g_ref[nz] - 1) <= G_RTOL)
-    rho_ref, cov_ref = geo.coverage(r.cams, qc, ref_uvz, hc, hs, hv, 0.9)
-    assert np.array_equal(rho.cpu().numpy(), rho_ref.astype(np.float32))
-    assert np.array_equal(cov.cpu().numpy(), cov_ref)
+    g_ref, g_lo, g_hi = geo.overlap_bounds(r.cams, qc, qs, hc, hs, hv, 8)
+    assert (g_ref > 0).any()
+    check_g_bounds(g.cpu().numpy().astype(np.float64), g_ref, g_lo, g_hi)
+    n, n_lo, n_hi = geo.coverage_bounds(r.cams, qc, quvz, hc, hs, hv)
+    check_coverage_bounds(rho.cpu().numpy(), cov.cpu().numpy(), n, n_lo, n_hi, b, 0.9)

@@ -102,3 +102,42 @@ def test_coverage_fraction_and_threshold():
     assert rho.tolist() == [1.0, 0.8] and cov.tolist() == [1, 0]
     rho, cov = geo.coverage(cams, [0, 0], uvz, [0], [SLAB], [0], eta=0.9)
     assert rho.tolist() == [0.0, 0.0]
+
+
+# ---- marginal decisions: the count interval [n_lo, n_hi] ----
+
+def test_grid_points_on_a_face_are_marginal():
+    # G = 4: the query box's samples sit at x in {-3, -1, 1, 3}.  The history
+    # box (half extent 4) shifted by 1 has its face at x = -3: one plane of
+    # 16 samples lies exactly on it (inside by definition, |d| <= h), so the
+    # fp64 count is 64, but another precision may put those 16 either side.
+    n, lo, hi, vi, vr = geo.slab_iou_counts(cam(), SLAB, cam(C=(1.0, 0.0, 0.0)), SLAB, True, 4)
+    assert (n, lo, hi) == (64, 48, 64)
+    # moved a thousandth further the plane is clearly outside: no margin case
+    n, lo, hi, _, _ = geo.slab_iou_counts(cam(), SLAB, cam(C=(1.001, 0.0, 0.0)), SLAB, True, 4)
+    assert (n, lo, hi) == (48, 48, 48)
+    g, g_lo, g_hi = geo.overlap_bounds([cam(), cam(C=(1.0, 0.0, 0.0))], [0], [SLAB], [1],
+                                       [SLAB], [1], 4)
+    assert g_lo[0, 0] < g[0, 0] == g_hi[0, 0] == 1.0
+
+
+@pytest.mark.parametrize("G,k", [(4, 1), (8, 3)])
+def test_whole_cell_shifts_have_no_marginal_samples(G, k):
+    # samples sit half a cell from every face: the count is fixed
+    n, lo, hi, _, _ = geo.slab_iou_counts(cam(), SLAB, cam(C=(8.0 * k / G, 0.0, 0.0)), SLAB,
+                                          True, G)
+    assert n == lo == hi == G * G * (G - k)
+
+
+def test_token_on_a_rectangle_edge_is_marginal():
+    c = cam()
+    X = geo.token_world(c, 2.0, 3.0, 4.0)        # u exactly on the edge u0 = 2
+    inside, margin = geo.inside_margin(X, c, SLAB)
+    assert inside and margin == 0.0
+    uvz = np.array([[[2.0, 3.0, 4.0], [3.0, 3.0, 4.0], [1.5, 3.0, 4.0], [1.99, 3.0, 4.0]]],
+                   dtype=np.float32)
+    n, lo, hi = geo.coverage_bounds([c], [0], uvz, [0], [SLAB], [1])
+    # edge token: counted, marginal; (3, 3): inside by 1 token = 2 world
+    # units at depth 4; (1.5, 3) and (1.99, 3): outside by 0.5 and 0.01
+    # tokens (1 and 0.02 world units): both clear of the margin
+    assert (n[0], lo[0], hi[0]) == (2, 1, 2)

@@ -110,3 +110,59 @@ def test_sideways_whole_token_shift_and_recency():
     # the newest source gives every token one sample only: with k_warp = 2
     # nothing qualifies and the tokens stay holes
     assert np.all(osl.multiwarp([src, tgt], d_new, [0, 0], 1, H, W, s=1, k_warp=2) == 0)
+
+
+def test_block_tokens_on_a_hand_built_lattice():
+    # one frame (global frame 1) of H = 2, W = 4 tokens, s = 1; blocks of 4
+    # tokens in an arbitrary rank order.  Cell index = (f H + y) W + x.
+    H, W, b = 2, 4, 4
+    f = 1
+    order = [(1, 0), (0, 0), (0, 1), (1, 1),       # block 2: ranks 8..11 as (x, y)
+             (3, 1), (2, 1), (2, 0), (3, 0)]       # block 3: ranks 12..15
+    cell_of_rank = np.full(16, -1, dtype=np.int64)
+    for k, (x, y) in enumerate(order):
+        cell_of_rank[8 + k] = (f * H + y) * W + x
+    depth = np.array([[[1.0, 2.0, 0.0, 4.0],
+                       [5.0, -1.0, 7.0, 8.0]]], dtype=np.float32)
+    mask = np.array([[[1, 1, 1, 1], [1, 1, 1, 0]]], dtype=np.uint8)    # (3, 1) masked
+    conf = np.array([[[0.9, 0.4, 0.9, 0.9], [0.9, 0.9, 0.5, 0.9]]], dtype=np.float32)
+    out = osl.block_tokens(depth, conf, mask, cell_of_rank, H, W, b, frame_base=1,
+                           first_block=2, n_blocks=2, c_min=0.5)
+    # (x + 0.5, y + 0.5, depth), depth 0 when the sample is not reliable:
+    # (1, 0) conf 0.4 < 0.5; (1, 1) depth -1; (2, 0) depth 0; (3, 1) masked;
+    # (2, 1) conf exactly 0.5 is kept
+    want = [[[1.5, 0.5, 0.0], [0.5, 0.5, 1.0], [0.5, 1.5, 5.0], [1.5, 1.5, 0.0]],
+            [[3.5, 1.5, 0.0], [2.5, 1.5, 7.0], [2.5, 0.5, 0.0], [3.5, 0.5, 4.0]]]
+    assert out.dtype == np.float32 and out.tolist() == want
+    # no confidence or mask given: only the depth decides
+    out = osl.block_tokens(depth, None, None, cell_of_rank, H, W, b, 1, 2, 2)
+    assert out[0, 0, 2] == 2.0 and out[1, 0, 2] == 8.0 and out[0, 3, 2] == 0.0
+
+
+def test_samples_landing_on_token_edges_are_unsure():
+    H, W, Z = 4, 8, 4.0
+    d = np.full((1, H, W), Z, dtype=np.float32)
+    # a sideways move of 0.5 world units at depth 4, fx = 4: half a token.
+    # Token centres x + 0.5 land on x exactly: every landing is on an edge.
+    src, tgt = cam(), cam(C=(0.5, 0.0, 0.0))
+    zq, unsure = osl.multiwarp_bounds([src, tgt], d, [0], 1, H, W, s=1, k_warp=1)
+    assert unsure.all()
+    # a quarter of a token: token x lands at x + 0.25, a quarter token from
+    # the nearest edge, in its own cell
+    zq, unsure = osl.multiwarp_bounds([src, cam(C=(0.25, 0.0, 0.0))], d, [0], 1, H, W, s=1,
+                                      k_warp=1)
+    assert not unsure.any()
+    assert np.all(zq == Z)
+
+
+def test_warp_sample_closed_form():
+    # forward move by 1 towards depth 4: depth 3, same pixel for the principal
+    # ray, and the landing cell with its distance to the nearest token edge
+    cell, depth, margin, cand = osl.warp_sample(cam(), cam(C=(0.0, 0.0, 1.0)), 4.5, 2.5, 4.0,
+                                                4, 8)
+    # u' = (4.5 - 4) * 4 / 3 + 4 = 4.666..., v' = (2.5 - 2) * 4 / 3 + 2 = 2.666...
+    assert cell == (4, 2) and depth == 3.0 and cand == [(4, 2)]
+    assert abs(margin - (1.0 / 3.0) * 3.0 / 4.0) < 1e-12
+    # behind the target camera: no landing
+    cell, depth, _, _ = osl.warp_sample(cam(), cam(C=(0.0, 0.0, 5.0)), 4.5, 2.5, 4.0, 4, 8)
+    assert cell is None and depth < 0
