@@ -65,6 +65,31 @@ def frame_curve(width: int, height: int) -> list:
 
 
 def _walk(cells, x, y, ax, ay, bx, by):
+    # The steps below are those of Jakub Cerveny's published generalised
+    # Hilbert ("gilbert") construction, which this function restates; that
+    # project is distributed under the BSD 2-Clause licence, whose notice is
+    # reproduced here:
+    #
+    #   Copyright (c) 2018, Jakub Cerveny.  All rights reserved.
+    #   Redistribution and use in source and binary forms, with or without
+    #   modification, are permitted provided that the following conditions
+    #   are met: 1. Redistributions of source code must retain the above
+    #   copyright notice, this list of conditions and the following
+    #   disclaimer.  2. Redistributions in binary form must reproduce the
+    #   above copyright notice, this list of conditions and the following
+    #   disclaimer in the documentation and/or other materials provided with
+    #   the distribution.
+    #   THIS SOFTWARE IS PROVIDED BY THE COPYRIGHT HOLDERS AND CONTRIBUTORS
+    #   "AS IS" AND ANY EXPRESS OR IMPLIED WARRANTIES, INCLUDING, BUT NOT
+    #   LIMITED TO, THE IMPLIED WARRANTIES OF MERCHANTABILITY AND FITNESS FOR
+    #   A PARTICULAR PURPOSE ARE DISCLAIMED.  IN NO EVENT SHALL THE COPYRIGHT
+    #   HOLDER OR CONTRIBUTORS BE LIABLE FOR ANY DIRECT, INDIRECT, INCIDENTAL,
+    #   SPECIAL, EXEMPLARY, OR CONSEQUENTIAL DAMAGES (INCLUDING, BUT NOT
+    #   LIMITED TO, PROCUREMENT OF SUBSTITUTE GOODS OR SERVICES; LOSS OF USE,
+    #   DATA, OR PROFITS; OR BUSINESS INTERRUPTION) HOWEVER CAUSED AND ON ANY
+    #   THEORY OF LIABILITY, WHETHER IN CONTRACT, STRICT LIABILITY, OR TORT
+    #   (INCLUDING NEGLIGENCE OR OTHERWISE) ARISING IN ANY WAY OUT OF THE USE
+    #   OF THIS SOFTWARE, EVEN IF ADVISED OF THE POSSIBILITY OF SUCH DAMAGE.
     n_major = abs(ax + ay)
     n_minor = abs(bx + by)
     ux, uy = _sign(ax), _sign(ay)   # unit step along the major edge
