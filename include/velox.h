@@ -32,7 +32,9 @@
  * - Every pointer argument is a DEVICE pointer, owned by the caller, unless
  *   the argument says "host".  The library never allocates, frees or keeps
  *   caller memory; it keeps no state between calls except a per-device
- *   cache of device attributes.
+ *   cache of device attributes and one exception: the fixed device array of
+ *   VELOX_NOALLOC_SCRATCH_BYTES and its cached address, used only by
+ *   velox_block_importance_noalloc.
  * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *   default stream) and may be issued from several host threads.
  * - Tensors are dense and contiguous in the layouts stated.  bf16 values are
@@ -217,8 +219,11 @@ VELOX_API velox_status velox_block_importance(const velox_bf16 *Q, const velox_b
  * array (H * (N + M) <= 131072 at d = 128); larger sizes return
  * VELOX_ERR_WORKSPACE before any launch.  The first call on each device
  * looks up the array's device address (cudaGetSymbolAddress, which may load
- * the library's device code); make that first call before any stream
- * capture.  Every call on a device shares the one array and leaves its
+ * the library's device code) and caches it for the device's current context;
+ * make that first call before any stream capture.  cudaDeviceReset (or
+ * anything else that replaces the device's primary context) discards the
+ * cache: the next call looks the address up again, so it too belongs before
+ * any capture.  Every call on a device shares the one array and leaves its
  * contents behind: calls that overlap on the GPU (other streams, unordered
  * host threads) race on it.
  */

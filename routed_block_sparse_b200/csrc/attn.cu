@@ -7,49 +7,66 @@
 // attention restricted to the tokens of the listed tiles, computed with the
 // FlashAttention online-softmax recurrence over tiles.
 //
-// sm_100a design: one CTA per (head, query block), one CTA per SM.  The
-// tiles of the route are split into two interleaved chains, even and odd,
-// each with its own S buffer and its own O accumulator in TMEM (4 x 128
-// columns) and its own softmax warpgroup with its own running max and row
-// sum, so two tiles are in their softmax at once; the epilogue merges the
-// two partial results (FlashAttention's split-KV merge, inside the CTA).
-// CTAs take rows in the order `row_order` gives (longest routes first, from
-// velox_route_schedule), so the last wave is made of short rows.
-//   warp 0      TMA producer: Q once, then K_0, V_0, K_1, V_1, ... of the
-//               route into a ring of 32 KB slots (128-byte swizzle, two
-//               64-channel boxes per tile).
-//   warp 1      TMEM allocator and the single tcgen05.mma issuer.  S_j =
-//               Q K_j^T (both operands from shared memory) goes into buffer
-//               j mod 2; once the softmax of tile j is done it issues
-//               O_{j mod 2} += P_j V_j (A = P from TMEM, B = V from shared
-//               memory) and, as soon as that has completed, S_{j+2} into the
-//               same buffer.
-//   warps 2-5   softmax of the even tiles, warps 6-9 of the odd tiles: one
-//               query row per thread (its TMEM lane).  Two TMEM reads of the
-//               S row (168 registers per thread do not hold the row and the
-//               rest): the three-input max, then 32 columns at a time the
-//               scaled exponent arguments and the row sum in packed fp32x2
-//               arithmetic, exponentials on MUFU,
-//               P_j packed to bf16 into the first 64 columns of its own S
-//               buffer (column t/2 holds elements t, t+1).  A chain's running
-//               max only moves (and its O is rescaled in TMEM, after its
-//               previous PV) when it grows by more than 2^8; a stale max is
-//               exact because the chain's O and row sum use the same one.
-//               Epilogue: the two chains exchange (max, sum) per row through
-//               shared memory; thread (row, chain c) writes channels
-//               64c..64c+63 of O = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / l, and lse.
+// sm_100a design: one CTA per (head, query block), one CTA per SM, 384
+// threads in three warpgroups.  CTAs take rows in the order `row_order`
+// gives (longest routes first, from velox_route_schedule), so the last wave
+// is made of short rows.
+//
+// TMEM (512 columns): two S buffers (fp32, 128 columns each), one O
+// accumulator (fp32, 128) and two P buffers (bf16 pairs, 64 each).  Tile j
+// has its S in buffer j mod 2 and its P in buffer j mod 2; the softmax of
+// even and odd tiles runs in two warpgroups at once.  Because P has buffers
+// of its own, S_{j+2} can be issued as soon as the softmax of tile j has
+// loaded S_j into registers: the score product of a tile overlaps the
+// softmax of the tile before it in the same buffer, and the per-buffer chain
+// S -> softmax -> PV -> S is broken.
+//
+// All tiles accumulate into the one O, so all of them use one per-row
+// reference max: tile j takes the reference of tile j - 1 (handed over per
+// row through shared memory) and raises it only when its own row max exceeds
+// it by more than 2^8 (a stale reference is exact: P and the row sums use
+// the same one).  When it rises, O is rescaled in TMEM between PV_{j-1} and
+// PV_j by the softmax threads of tile j.
+//   warpgroup 0 (56 registers per thread after setmaxnreg), one thread per
+//   warp active:
+//     warp 0    TMA producer of Q and of the route's K tiles, warp 2 of its V
+//               tiles, into two rings of 32 KB slots (128-byte swizzle, two
+//               64-channel boxes per tile): a K slot is freed by its score
+//               product, a V slot by its PV, so neither stream waits on the
+//               other.
+//     warp 1    TMEM allocator and issuer of the score products: S_{j+2} =
+//               Q K_{j+2}^T once the softmax of tile j has read S_j.
+//     warp 3    issuer of O += P_j V_j (A = P from TMEM, B = V from shared
+//               memory) once P_j is written.  Two issuing threads: each
+//               tcgen05.commit tracks only its own thread's products, so a
+//               PV never waits behind a K load and S never behind a PV.
+//   warpgroups 1 and 2 (224 registers per thread): softmax of the even and
+//     of the odd tiles, one query row per thread (its TMEM lane): the whole
+//     128-column S row read from TMEM in one go, the row max, the reference
+//     hand-over, exponent arguments and the row sum in packed fp32x2
+//     arithmetic, exponentials on MUFU (a share of them, set by kPolyPairs,
+//     by a cubic on the FMA pipe), P packed to bf16 into its P buffer
+//     (column t/2 holds elements t, t+1).  Each warpgroup keeps its row sums
+//     in the reference of its own last tile; the epilogue brings both to the
+//     final reference and writes O / l and the lse.
 // A pre-pass compacts the route into shared memory, skipping ids outside
 // [0, M) and repeats (flagged in dev_status).
 //
 // Two-phase form (digest, "Reproducibility": the two-phase tile loop): after
 // the routed history tiles the same loop visits the n_cur tiles of the
-// current chunk's own K/V (separate tensors), alternating between the two
-// chains like any other tiles, so the merged normaliser covers both phases.
+// current chunk's own K/V (separate tensors), like any other tiles, so the
+// one softmax covers both phases.
 #include <cudaTypedefs.h>
 
 #include <mutex>
 
 #include "common.cuh"
+
+// Of every 8 exponent pairs of a row, this many are computed by the cubic on
+// the FMA pipe instead of MUFU (0..8).
+#ifndef VELOX_ATTN_POLY_PAIRS
+#define VELOX_ATTN_POLY_PAIRS 0
+#endif
 
 namespace velox {
 namespace {
@@ -57,25 +74,38 @@ namespace {
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // tokens per KV tile
 constexpr int D = 128;   // head dim
-constexpr int kThreads = 320;  // TMA warp, MMA warp, 2 x 4 softmax warps
-constexpr int kChainThreads = 128;  // softmax threads of one chain
+constexpr int kThreads = 384;       // 3 warpgroups
+constexpr int kChainThreads = 128;  // softmax threads of one warpgroup
 constexpr int kSoftThreads = 256;
+// register split: the launch gives every thread kRegsLaunch; warpgroup 0
+// hands registers back and the two softmax warpgroups take them
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsCtl = 56;
+constexpr int kRegsSoft = 224;
+static_assert(128 * kRegsCtl + 2 * 128 * kRegsSoft <= kThreads * kRegsLaunch,
+              "setmaxnreg split exceeds the registers the block is launched with");
+constexpr int kPolyPairs = VELOX_ATTN_POLY_PAIRS;
+static_assert(kPolyPairs >= 0 && kPolyPairs <= 8, "kPolyPairs out of range");
 constexpr uint32_t kTileBytes = BN * D * 2;      // 32 KB
 constexpr uint32_t kHalfBytes = kTileBytes / 2;  // one 64-channel box
 constexpr int kMaxRoute = VELOX_MAX_ROUTE;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kSBufs = 2;         // S/P buffers in TMEM (one per chain), columns 0 and 128
-constexpr uint32_t kColO = 256;   // O accumulators (fp32, 128 columns each), 256 and 384
-constexpr int kMaxSlots = 6;      // K/V ring slots of 32 KB
+constexpr int kBufs = 2;             // S and P buffers (tile j uses buffer j mod 2)
+constexpr uint32_t kColS = 0;        // S buffers: columns 0 and 128
+constexpr uint32_t kColO = 256;      // O accumulator: columns 256..383
+constexpr uint32_t kColP = 384;      // P buffers: columns 384 and 448
+constexpr int kMaxSlots = 6;         // K/V ring slots of 32 KB
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest tolerated growth
 
 // shared-memory layout (offsets from a 1024-byte aligned base)
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffRing = kOffQ + kTileBytes;
-// barriers, misc and the dynamic tail follow the ring (offset set at launch)
-// q_full, the K/V ring, s_full/p_full/pv_done per chain, x_fin, mma_done
-constexpr uint32_t kNumBars = 1 + 2 * kMaxSlots + 3 * kSBufs + 1 + 1;
+// barriers, misc, the reference hand-over and the route list follow the ring
+// (offsets set at launch).  Barriers: q_full, the K/V ring (full, empty),
+// per buffer s_full / s_free / p_full / pv_done / ref_full, x_fin, mma_done.
+constexpr uint32_t kNumBars = 1 + 2 * kMaxSlots + 5 * kBufs + 1 + 1;
 constexpr uint32_t kMiscBytes = 64;
+constexpr uint32_t kRefBytes = BM * 4;  // one fp32 reference per row
 constexpr uint32_t kSmemLimit = 227 * 1024;
 
 struct AttnArgs {
@@ -91,10 +121,10 @@ struct AttnArgs {
   uint16_t *O;
   float *lse;
   int32_t *dev_status;
-  int nslot;              // K/V ring slots in use (4..kMaxSlots)
+  int nslot;              // ring slots in use (4 or 6): half K, half V
   uint32_t bar_offset;    // byte offset of the barriers from the aligned base
+  uint32_t ref_offset;    // reference hand-over (fp32 per row)
   uint32_t list_offset;   // route list (uint16)
-  uint32_t bits_offset;   // id bitmap (uint32)
 };
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_saddr, int k) {
@@ -124,7 +154,34 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
 }
 
-// 10 warps: three share a scheduler, whose 16 K registers then allow 168 each
+// 2^x for a pair of fp32 values on the FMA pipe: x = k + f with k the
+// nearest integer (the 1.5 * 2^23 shifter puts k in the low mantissa bits)
+// and f in [-0.5, 0.5]; 2^f from a cubic fitted to it here by iterated
+// weighted least squares for the smallest relative error on [-0.5, 0.5]
+// (7.5e-5, far below the bf16 rounding of P); k is added to the exponent
+// field.  Arguments are clamped at -125 so the result stays a normal number
+// (2^-125 instead of a smaller value: an absolute error below 3e-38 against
+// a row sum of at least 2^-8).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261114f, c3 = 0.055171669f;
+  float a, b;
+  f2unpack(x2, a, b);
+  const uint64_t x = f2pack(fmaxf(a, -125.0f), fmaxf(b, -125.0f));
+  const uint64_t t = fadd2(x, f2pack(kShift, kShift));
+  const uint64_t kf = fadd2(t, f2pack(-kShift, -kShift));
+  const uint64_t f = ffma2(kf, f2pack(-1.0f, -1.0f), x);
+  uint64_t p = ffma2(f2pack(c3, c3), f, f2pack(c2, c2));
+  p = ffma2(p, f, f2pack(c1, c1));
+  p = ffma2(p, f, f2pack(c0, c0));
+  float p0, p1, t0, t1;
+  f2unpack(p, p0, p1);
+  f2unpack(t, t0, t1);
+  const float r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  const float r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+  return f2pack(r0, r1);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
@@ -138,17 +195,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *q_full = bar;
   uint64_t *slot_full = q_full + 1;
   uint64_t *slot_empty = slot_full + kMaxSlots;
-  uint64_t *s_full = slot_empty + kMaxSlots;   // [chain]
-  uint64_t *p_full = s_full + kSBufs;          // [chain]
-  uint64_t *pv_done = p_full + kSBufs;         // [chain]
-  uint64_t *x_fin = pv_done + kSBufs;          // both chains' (max, sum) written
-  uint64_t *mma_done = x_fin + 1;
+  uint64_t *s_full = slot_empty + kMaxSlots;  // [buffer]: S_j written
+  uint64_t *s_free = s_full + kBufs;          // [buffer]: S_j read by its softmax
+  uint64_t *p_full = s_free + kBufs;          // [buffer]: P_j written
+  uint64_t *pv_done = p_full + kBufs;         // [buffer]: PV_j (and all before) done
+  uint64_t *ref_full = pv_done + kBufs;       // [buffer]: reference of tile j handed over
+  uint64_t *x_fin = ref_full + kBufs;         // both warpgroups' row sums written
+  uint64_t *mma_done = x_fin + 1;             // every MMA of the CTA done
   uint8_t *misc = base + a.bar_offset + kNumBars * 8;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(misc);
   int *s_nvalid = reinterpret_cast<int *>(misc + 4);
   volatile int *s_abort = reinterpret_cast<volatile int *>(misc + 8);
+  float *refx = reinterpret_cast<float *>(base + a.ref_offset);
   uint16_t *tiles = reinterpret_cast<uint16_t *>(base + a.list_offset);
-  uint32_t *bits = reinterpret_cast<uint32_t *>(base + a.bits_offset);
+  // the id bitmap of the route compaction lives in the ring, idle until the
+  // first load
+  uint32_t *bits = reinterpret_cast<uint32_t *>(ring);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = a.row_order ? a.row_order[blockIdx.x] : (int)blockIdx.x;
@@ -168,13 +230,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&slot_full[s], 1);
       mbar_init(&slot_empty[s], 1);
     }
-    for (int b = 0; b < kSBufs; ++b) {
+    for (int b = 0; b < kBufs; ++b) {
       mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], kChainThreads);
       mbar_init(&p_full[b], kChainThreads);
       mbar_init(&pv_done[b], 1);
+      mbar_init(&ref_full[b], kChainThreads);
     }
     mbar_init(x_fin, kSoftThreads);
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, 2);  // one commit from each MMA-issuing thread
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -222,204 +286,243 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   tc_fence_before();
-  __syncthreads();
+  __syncthreads();  // the bitmap is dead from here on: the ring may be loaded
   tc_fence_after();
   const int n_hist = *s_nvalid;
   const int n = n_hist + a.n_cur;  // tiles of both phases
   const uint32_t tmem = *s_tmem;
+  const int wg = warp >> 2;
 
-  if (warp == 0) {
-    // ================= TMA producer =================
-    if (lane == 0 && n > 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      if (a.n_cur > 0) {
-        prefetch_tmap(&tmKc);
-        prefetch_tmap(&tmVc);
+  if (wg == 0) {
+    regs_dec<kRegsCtl>();
+    // K and V have rings of their own (kk slots each): a K slot is freed by
+    // its score product, a V slot by its PV, so K loads run ahead of the
+    // score products without waiting for the PVs and the other way round.
+    const int kk = nslot / 2;
+    if (warp == 0 || warp == 2) {
+      // ================= TMA producers: warp 0 K (and Q), warp 2 V =================
+      const bool is_k = warp == 0;
+      if (lane == 0 && n > 0) {
+        const CUtensorMap *hist_map = is_k ? &tmK : &tmV;
+        const CUtensorMap *cur_map = is_k ? &tmKc : &tmVc;
+        prefetch_tmap(hist_map);
+        if (a.n_cur > 0) prefetch_tmap(cur_map);
+        // the ring held the compaction bitmap (generic-proxy writes) just
+        // before these asynchronous copies overwrite it
+        fence_proxy_async_smem();
+        if (is_k) {
+          prefetch_tmap(&tmQ);
+          mbar_arrive_expect_tx(q_full, kTileBytes);
+          tma_load_3d(sQ, &tmQ, q_full, 0, i * BM, h);
+          tma_load_3d(sQ + kHalfBytes, &tmQ, q_full, 64, i * BM, h);
+        }
+        const int s0 = is_k ? 0 : kk;  // first slot of this ring
+        int issued = 0;
+        for (int j = 0; j < n; ++j) {
+          const int s = s0 + j % kk;
+          const uint32_t use = j / kk;
+          if (!mbar_wait(&slot_empty[s], (use & 1) ^ 1, s_abort)) break;
+          const bool hist = j < n_hist;
+          const int tile = hist ? (dense ? j : tiles[j]) : j - n_hist;
+          const CUtensorMap *map = hist ? hist_map : cur_map;
+          uint8_t *dst = ring + s * kTileBytes;
+          mbar_arrive_expect_tx(&slot_full[s], kTileBytes);
+          tma_load_3d(dst, map, &slot_full[s], 0, tile * BN, h);
+          tma_load_3d(dst + kHalfBytes, map, &slot_full[s], 64, tile * BN, h);
+          issued = j + 1;
+        }
+        if (*s_abort) {
+          // let the copies already in flight land before the CTA goes away
+          // (each wait is bounded by the same time limit)
+          volatile int never = 0;
+          if (is_k) mbar_wait(q_full, 0, &never);
+          for (int j = issued - kk < 0 ? 0 : issued - kk; j < issued; ++j) {
+            never = 0;
+            mbar_wait(&slot_full[s0 + j % kk], (j / kk) & 1, &never);
+          }
+        }
       }
-      mbar_arrive_expect_tx(q_full, kTileBytes);
-      tma_load_3d(sQ, &tmQ, q_full, 0, i * BM, h);
-      tma_load_3d(sQ + kHalfBytes, &tmQ, q_full, 64, i * BM, h);
-      int issued = 0;
-      for (int li = 0; li < 2 * n; ++li) {  // load li: K_{li/2} (even) or V_{li/2} (odd)
-        const int s = li % nslot;
-        const uint32_t use = li / nslot;
-        if (!mbar_wait(&slot_empty[s], (use & 1) ^ 1, s_abort)) break;
-        const int j = li >> 1;
-        const bool hist = j < n_hist;
-        const int tile = hist ? (dense ? j : tiles[j]) : j - n_hist;
-        const CUtensorMap *map = (li & 1) ? (hist ? &tmV : &tmVc) : (hist ? &tmK : &tmKc);
-        uint8_t *dst = ring + s * kTileBytes;
-        mbar_arrive_expect_tx(&slot_full[s], kTileBytes);
-        tma_load_3d(dst, map, &slot_full[s], 0, tile * BN, h);
-        tma_load_3d(dst + kHalfBytes, map, &slot_full[s], 64, tile * BN, h);
-        issued = li + 1;
-      }
-      if (*s_abort) {
-        // let the copies already in flight land before the CTA goes away
-        // (each wait is bounded by the same time limit)
+    } else {
+      // ========== MMA issuers: warp 1 the score products, warp 3 the PVs ==========
+      // Each thread commits only its own products, so S_{j+2} never waits
+      // behind a PV and a PV never waits behind a K load; mma_done takes one
+      // arrival from each.
+      const bool is_s = warp == 1;
+      if (lane == 0 && n > 0) {
+        const uint32_t ra = smem_u32(ring);
+        bool ok = true;
+        if (is_s) {
+          constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false);
+          const uint32_t qa = smem_u32(sQ);
+          // S_j = Q K_j^T into S buffer j mod 2
+          auto issue_s = [&](int j) -> bool {
+            const int s = j % kk;
+            if (!mbar_wait(&slot_full[s], (j / kk) & 1, s_abort)) return false;
+            tc_fence_after();
+            const uint32_t ka = ra + s * kTileBytes;
+            const uint32_t sbuf = tmem + kColS + (j & 1) * BN;
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k)
+              mma_bf16_ss(sbuf, kmajor_desc(qa, k), kmajor_desc(ka, k), idS, k > 0);
+            tc_commit(&s_full[j & 1]);
+            tc_commit(&slot_empty[s]);
+            return true;
+          };
+          ok = mbar_wait(q_full, 0, s_abort) && issue_s(0);
+          if (ok && n > 1) ok = issue_s(1);
+          // S_{j+2} goes into the buffer of S_j once its softmax has read it
+          for (int j = 0; ok && j + 2 < n; ++j)
+            ok = mbar_wait(&s_free[j & 1], (j >> 1) & 1, s_abort) && issue_s(j + 2);
+        } else {
+          constexpr uint32_t idPV = idesc_bf16_f32(BM, D, true);
+          // O += P_j V_j, P_j in P buffer j mod 2 (A from TMEM)
+          for (int j = 0; ok && j < n; ++j) {
+            const int b = j & 1, s = kk + j % kk;
+            ok = mbar_wait(&p_full[b], (j >> 1) & 1, s_abort) &&
+                 mbar_wait(&slot_full[s], (j / kk) & 1, s_abort);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t va = ra + s * kTileBytes;
+            const uint32_t pb = tmem + kColP + b * (BN / 2);
+#pragma unroll
+            for (int k = 0; k < BN / 16; ++k)
+              mma_bf16_ts(tmem + kColO, pb + k * 8, vmn_desc(va, k), idPV, (j > 0 || k > 0));
+            tc_commit(&pv_done[b]);
+            tc_commit(&slot_empty[s]);
+          }
+        }
+        // every product this thread issued must be complete before TMEM is
+        // released (and before the epilogue reads O and reuses the ring)
+        tc_commit(mma_done);
         volatile int never = 0;
-        mbar_wait(q_full, 0, &never);
-        for (int li = issued - nslot < 0 ? 0 : issued - nslot; li < issued; ++li) {
-          never = 0;
-          mbar_wait(&slot_full[li % nslot], (li / nslot) & 1, &never);
-        }
+        mbar_wait(mma_done, 0, &never);
       }
-    }
-  } else if (warp == 1) {
-    // ================= MMA issuer =================
-    if (lane == 0 && n > 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false);
-      constexpr uint32_t idPV = idesc_bf16_f32(BM, D, true);
-      const uint32_t qa = smem_u32(sQ), ra = smem_u32(ring);
-      auto issue_s = [&](int j) -> bool {
-        const int li = 2 * j, s = li % nslot;
-        if (!mbar_wait(&slot_full[s], (li / nslot) & 1, s_abort)) return false;
-        tc_fence_after();
-        const uint32_t ka = ra + s * kTileBytes;
-        const uint32_t sb = tmem + (j & 1) * BN;
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-          mma_bf16_ss(sb, kmajor_desc(qa, k), kmajor_desc(ka, k), idS, k > 0);
-        tc_commit(&s_full[j & 1]);
-        tc_commit(&slot_empty[s]);
-        return true;
-      };
-      bool ok = mbar_wait(q_full, 0, s_abort);
-      if (ok) ok = issue_s(0);
-      if (ok && n > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < n; ++j) {
-        const int b = j & 1;  // chain
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(&p_full[b], ph, s_abort)) break;
-        const int li = 2 * j + 1, s = li % nslot;
-        if (!mbar_wait(&slot_full[s], (li / nslot) & 1, s_abort)) break;
-        tc_fence_after();
-        const uint32_t va = ra + s * kTileBytes;
-        const uint32_t pb = tmem + b * BN;  // P_j: first 64 columns of its S buffer
-#pragma unroll
-        for (int k = 0; k < BN / 16; ++k)
-          mma_bf16_ts(tmem + kColO + b * D, pb + k * 8, vmn_desc(va, k), idPV, (j >= 2 || k > 0));
-        tc_commit(&pv_done[b]);
-        tc_commit(&slot_empty[s]);
-        if (j + 2 < n) {
-          // S_{j+2} goes into the buffer P_j occupies: PV_j must be done
-          if (!mbar_wait(&pv_done[b], ph, s_abort)) break;
-          if (!issue_s(j + 2)) break;
-        }
-      }
-      // all issued MMAs must be complete before TMEM is released
-      tc_commit(mma_done);
-      volatile int never = 0;
-      mbar_wait(mma_done, 0, &never);
     }
   } else {
-    // ================= softmax / epilogue (warps 2..9) =================
+    regs_inc<kRegsSoft>();
+    // ================= softmax / epilogue (warpgroups 1, 2) =================
     const int quarter = warp & 3;
-    const int ch = (warp - 2) >> 2;     // chain: tiles j with j % 2 == ch
+    const int ch = wg - 1;              // tiles j with j % 2 == ch
     const int r = quarter * 32 + lane;  // query row within the tile = TMEM lane
     const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t sb = trow + ch * BN;                 // this chain's S buffer
-    const uint32_t ob = trow + kColO + ch * D;          // this chain's O
+    const uint32_t sb = trow + kColS + ch * BN;        // this warpgroup's S buffer
+    const uint32_t pb = trow + kColP + ch * (BN / 2);  // this warpgroup's P buffer
+    const uint32_t ob = trow + kColO;                  // the O accumulator
     const float c = a.scale_log2;
-    float m_run = -INFINITY, l = 0.f;
+    float ref_own = -INFINITY;  // reference of this warpgroup's last tile
+    float l = 0.f;              // row sum of this warpgroup's tiles, in ref_own
     bool ok = true;
-    int last = -1;  // this chain's last tile
     for (int j = ch; j < n; j += 2) {
       const uint32_t ph = (j >> 1) & 1;
       if (!warp_wait(&s_full[ch], ph, s_abort)) { ok = false; break; }
       tc_fence_after();
-      // two passes over the S row (the register file holds 168 per thread):
-      // the max, then the exponentials 32 columns at a time
+      // the whole S row in registers: one TMEM round trip, then the buffer
+      // is free for S_{j+2}
+      uint32_t sv[128];
+      tmem_ld32(sb, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(sb + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_ld32(sb + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+      tmem_ld32(sb + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+      tmem_wait_ld();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&sv[32 * q]));
+      tc_fence_before();
+      mbar_arrive(&s_free[ch]);
       float mx[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t sv[64];
-        tmem_ld32(sb + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(sb + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_wait_ld();
-#pragma unroll
-        for (int k = 0; k < 32; ++k)
-          mx[k & 7] = fmax3(mx[k & 7], __uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1]));
-      }
+      for (int k = 0; k < 64; ++k)
+        mx[k & 7] = fmax3(mx[k & 7], __uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1]));
       const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
-                             fmaxf(mx[6], mx[7]));
-      const float m_cand = fmaxf(m_run, mt * c);
-      const bool grow = m_cand > m_run + kRescaleThreshold;  // always on the chain's first tile
-      const float m_use = grow ? m_cand : m_run;
-      const float alpha = fast_exp2(m_run - m_use);  // 1 if kept, 0 on the first tile
-      if (last >= 0 && __any_sync(0xffffffffu, grow)) {
-        // move this chain's O to the new max: its previous PV must be done
-        if (!warp_wait(&pv_done[ch], (last >> 1) & 1, s_abort)) { ok = false; break; }
+                             fmaxf(mx[6], mx[7])) * c;
+      // reference hand-over: tile j - 1 (the other warpgroup) wrote its
+      // reference to refx[r]; this tile raises it only on growth above 2^8
+      float ref_prev = -INFINITY;
+      if (j > 0) {
+        if (!warp_wait(&ref_full[ch ^ 1], ((j - 1) >> 1) & 1, s_abort)) { ok = false; break; }
+        ref_prev = refx[r];
+      }
+      const bool grow = mt > ref_prev + kRescaleThreshold;  // always on tile 0
+      const float ref = grow ? mt : ref_prev;
+      if (j + 1 < n) {
+        refx[r] = ref;  // read by tile j + 1 only after this arrival
+        mbar_arrive(&ref_full[ch]);
+      }
+      // P buffer reuse: PV_{j-2} (this buffer's last reader) must be done;
+      // that also puts every PV before it behind us
+      if (j >= 2 && !warp_wait(&pv_done[ch], ((j - 2) >> 1) & 1, s_abort)) { ok = false; break; }
+      // O rescale when the reference grew: after PV_{j-1}, before PV_j
+      if (j >= 1 && __any_sync(0xffffffffu, grow)) {
+        if (!warp_wait(&pv_done[ch ^ 1], ((j - 1) >> 1) & 1, s_abort)) { ok = false; break; }
         tc_fence_after();
+        const float alpha = fast_exp2(ref_prev - ref);  // 1 on rows that kept theirs
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t ov[32];
           tmem_ld32(ob + cc * 32, ov);
           tmem_wait_ld();
+          reg_fence(ov);
 #pragma unroll
           for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
           tmem_st32(ob + cc * 32, ov);
         }
       }
-      // exponentials (arguments and row sum in packed pairs); P_j into the
-      // first 64 columns of its S buffer: column t/2 holds elements t, t+1
+      // exponentials (arguments and row sum in packed pairs); P_j packed to
+      // bf16 into its buffer, 16 columns at a time: column t/2 holds
+      // elements t, t+1
       uint64_t sum2[2] = {0ull, 0ull};
-      const uint64_t c2 = f2pack(c, c), nm2 = f2pack(-m_use, -m_use);
+      const uint64_t c2 = f2pack(c, c), nr2 = f2pack(-ref, -ref);
 #pragma unroll
-      for (int qt = 0; qt < 4; ++qt) {  // S columns 32qt.. -> P columns 16qt.. (already read)
-        uint32_t sv[32];
-        tmem_ld32(sb + qt * 32, sv);
-        tmem_wait_ld();
+      for (int qt = 0; qt < 4; ++qt) {
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const uint64_t x2 = ffma2(f2pack(__uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1])),
-                                    c2, nm2);
-          float x0, x1;
-          f2unpack(x2, x0, x1);
-          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-          sum2[k & 1] = fadd2(sum2[k & 1], f2pack(p0, p1));
+          const int e = qt * 16 + k;  // pair index within the row
+          const uint64_t x2 =
+              ffma2(f2pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), c2, nr2);
+          uint64_t p2;
+          if ((e & 7) < kPolyPairs) {
+            p2 = exp2_poly2(x2);
+          } else {
+            float x0, x1;
+            f2unpack(x2, x0, x1);
+            p2 = f2pack(fast_exp2(x0), fast_exp2(x1));
+          }
+          sum2[k & 1] = fadd2(sum2[k & 1], p2);
+          float p0, p1;
+          f2unpack(p2, p0, p1);
           pk[k] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(sb + qt * 16, pk);
+        tmem_st16(pb + qt * 16, pk);
       }
       float sa, sb2;
       f2unpack(fadd2(sum2[0], sum2[1]), sa, sb2);
+      // this warpgroup's row sum moves to the new reference
+      l = l * fast_exp2(ref_own - ref) + (sa + sb2);  // 0 * 0 on the first tile
+      ref_own = ref;
       tmem_wait_st();
-      l = l * alpha + (sa + sb2);
-      m_run = m_use;
-      last = j;
       tc_fence_before();
       mbar_arrive(&p_full[ch]);
     }
-    // epilogue: merge the two chains.  Both chains' last PVs must be done
-    // before either O is read; (max, sum) per row go through shared memory
-    // (the ring, idle once every PV is done).
+    // epilogue: every MMA must be done before O is read and before the ring
+    // (idle from then on) takes the row-sum exchange; mma_done completes once
+    // per CTA, so the wait cannot meet an older phase.
     bool have = ok && n > 0;
-    if (have) {
-      for (int cc = 0; cc < 2 && cc < n; ++cc) {
-        const int lc = ((n - 1) & 1) == cc ? n - 1 : n - 2;  // chain cc's last tile
-        if (!mbar_wait(&pv_done[cc], (lc >> 1) & 1, s_abort)) { have = false; break; }
-      }
-    }
-    float *xm = reinterpret_cast<float *>(ring);  // [chain][2][128]: max, sum
-    xm[(ch * 2 + 0) * BM + r] = m_run;
+    if (have && !mbar_wait(mma_done, 0, s_abort)) have = false;
+    float *xm = reinterpret_cast<float *>(ring);  // [warpgroup][2][128]: reference, sum
+    xm[(ch * 2 + 0) * BM + r] = ref_own;
     xm[(ch * 2 + 1) * BM + r] = l;
     mbar_arrive(x_fin);
     const bool fin_ok = mbar_wait(x_fin, 0, s_abort);
-    const float mo = xm[((ch ^ 1) * 2 + 0) * BM + r];
-    const float lo = xm[((ch ^ 1) * 2 + 1) * BM + r];
-    const float m0 = ch == 0 ? m_run : mo, m1 = ch == 0 ? mo : m_run;
-    const float l0 = ch == 0 ? l : lo, l1 = ch == 0 ? lo : l;
-    const float mm = fmaxf(m0, m1);
-    // a chain without tiles has max -inf and sum 0: weight 0, O never read
-    const float w0 = n > 0 ? fast_exp2(m0 - mm) : 0.f;
-    const float w1 = n > 1 ? fast_exp2(m1 - mm) : 0.f;
-    const float l_row = l0 * w0 + l1 * w1;
+    const float ref_o = xm[((ch ^ 1) * 2 + 0) * BM + r];
+    const float l_o = xm[((ch ^ 1) * 2 + 1) * BM + r];
+    // O is in the reference of the last tile, the larger of the two
+    // (references only grow); a warpgroup without tiles has sum 0
+    const float ref_fin = fmaxf(ref_own, ref_o);
+    const float w_own = l > 0.f ? fast_exp2(ref_own - ref_fin) : 0.f;
+    const float w_o = l_o > 0.f ? fast_exp2(ref_o - ref_fin) : 0.f;
+    const float l_row = l * w_own + l_o * w_o;
     // tcgen05.ld is warp-collective: decide once for the whole warp
     const bool good = __all_sync(0xffffffffu, have && fin_ok && !*s_abort);
     tc_fence_after();
@@ -427,26 +530,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint16_t *orow = a.O + ((size_t)row * BM + r) * D + ch * 64;
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
-      uint32_t o0[16], o1[16];
+      uint32_t o0[16];
       if (good) {
-        tmem_ld16(trow + kColO + ch * 64 + cc * 16, o0);
-        if (n > 1) tmem_ld16(trow + kColO + D + ch * 64 + cc * 16, o1);
+        tmem_ld16(ob + ch * 64 + cc * 16, o0);
         tmem_wait_ld();
+        reg_fence(o0);
       } else {
 #pragma unroll
         for (int k = 0; k < 16; ++k) o0[k] = 0u;
       }
-      if (!good || n < 2) {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) o1[k] = 0u;
-      }
-      const float s0 = w0 * inv, s1 = w1 * inv;
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         float v[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          v[e] = __uint_as_float(o0[8 * q + e]) * s0 + __uint_as_float(o1[8 * q + e]) * s1;
+        for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(o0[8 * q + e]) * inv;
         uint4 u;
         u.x = pack_bf16x2(v[0], v[1]);
         u.y = pack_bf16x2(v[2], v[3]);
@@ -456,7 +553,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (a.lse && ch == 0)
-      a.lse[(size_t)row * BM + r] = good ? (mm + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
+      a.lse[(size_t)row * BM + r] =
+          good ? (ref_fin + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
   }
 
   if (*s_abort && threadIdx.x == 0) flag_error(a.dev_status, VELOX_DEV_WAIT_TIMEOUT);
@@ -531,22 +629,33 @@ cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
   a.O = O;
   a.lse = lse;
   a.dev_status = dev_status;
-  // tail after the ring: barriers, misc, route list (uint16), id bitmap
+  // tail after the ring: barriers, misc, the reference hand-over, the route
+  // list (uint16).  The compaction bitmap (M bits) lives in the ring.
   const uint32_t list_bytes = route_ids ? ((uint32_t)R_max * 2u + 15u) & ~15u : 0u;
-  const uint32_t bits_bytes = route_ids ? (uint32_t)((M + 31) / 32) * 4u : 0u;
-  const uint32_t tail = kNumBars * 8 + kMiscBytes + list_bytes + bits_bytes;
+  const uint32_t tail = kNumBars * 8 + kMiscBytes + kRefBytes + list_bytes;
   int nslot = kMaxSlots;
   while (nslot > 4 && kOffRing + nslot * kTileBytes + tail + 1024 > kSmemLimit) --nslot;
-  // loads go K_0, V_0, K_1, V_1, ... round the ring; load li reuses the slot
-  // of load li - nslot.  With an odd count K_{j+3} would reuse V_j's slot and
-  // could not start before PV_j, just when S_{j+3} is wanted: keep it even.
+  // K and V rings of nslot / 2 slots each
   nslot &= ~1;
   a.nslot = nslot;
   a.bar_offset = kOffRing + nslot * kTileBytes;
-  a.list_offset = a.bar_offset + kNumBars * 8 + kMiscBytes;
-  a.bits_offset = a.list_offset + list_bytes;
-  const size_t smem = (size_t)a.bits_offset + bits_bytes + 1024;  // + alignment slack
-  if (smem > kSmemLimit) return cudaErrorInvalidConfiguration;
+  a.ref_offset = a.bar_offset + kNumBars * 8 + kMiscBytes;
+  a.list_offset = a.ref_offset + kRefBytes;
+  const size_t smem = (size_t)a.list_offset + list_bytes + 1024;  // + alignment slack
+  if (smem > kSmemLimit || (size_t)nslot * kTileBytes < (size_t)(M + 31) / 32 * 4)
+    return cudaErrorInvalidConfiguration;
+  // The setmaxnreg split draws on the registers of the launch: refuse to
+  // launch a build whose per-thread count is below the one it was planned for
+  // (the softmax warpgroups would wait forever for registers).
+  static cudaError_t regs_ok = [] {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_kernel);
+    if (e != cudaSuccess) return e;
+    return fa.numRegs * kThreads >= 128 * kRegsCtl + 2 * 128 * kRegsSoft
+               ? cudaSuccess
+               : cudaErrorInvalidConfiguration;
+  }();
+  if (regs_ok != cudaSuccess) return regs_ok;
   cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;

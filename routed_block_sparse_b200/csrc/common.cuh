@@ -72,6 +72,19 @@ VELOX_DEVFN bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe: true once the phase of `parity` has completed.
+VELOX_DEVFN bool mbar_test(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 VELOX_DEVFN uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -120,6 +133,19 @@ VELOX_DEVFN void prefetch_tmap(const CUtensorMap *map) {
 // proxy (TMA, tensor core operand reads).
 VELOX_DEVFN void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ------------------------------------------------- register reallocation ---
+// setmaxnreg: executed by every thread of a warpgroup.  dec hands registers
+// back to the block's pool, inc takes them (waiting until they are free);
+// the sum over warpgroups must fit in what the block was launched with.
+template <uint32_t R>
+VELOX_DEVFN void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+VELOX_DEVFN void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
 }
 
 // -------------------------------------------------------------- tcgen05 ---
@@ -210,6 +236,23 @@ VELOX_DEVFN void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
       : "memory");
 }
 VELOX_DEVFN void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Register fences for the destinations of tcgen05.ld: the load writes its
+// registers asynchronously, and nothing in the C++ data flow ties their uses
+// to the later tcgen05.wait::ld.  An empty volatile asm that "redefines" the
+// registers, placed right after the wait, makes every use depend on it.
+VELOX_DEVFN void reg_fence(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
+VELOX_DEVFN void reg_fence(uint32_t (&r)[32]) {
+  reg_fence(*reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+  reg_fence(*reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+}
 VELOX_DEVFN void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor (tcgen05), 128-byte swizzle.

@@ -10,12 +10,19 @@
 // The array is a file-scope __device__ variable, so every GPU that loads the
 // library holds it (kNoAllocScratchBytes) until the process exits.  In host
 // code its name is only a host-side stand-in; its device address is looked up
-// once per device with cudaGetSymbolAddress, on the first call made while
-// that device is current, and passed to the kernels.  Nothing in the array
-// must start at zero (the pooling kernel writes every mean before the logit
-// kernel reads it), so no call clears it.  All calls on a device share the
-// one array: calls that overlap on the GPU (other streams, unordered host
+// with cudaGetSymbolAddress on the first call made while that device is
+// current, cached, and passed to the kernels.  The cache is keyed on the
+// device's current context (its driver-assigned context id, never reused in a
+// process): after cudaDeviceReset, or anything else that replaces the
+// device's primary context, the module is loaded again and the array may sit
+// at another address, so the next call looks it up again instead of handing
+// the kernels a stale pointer.  A failed lookup is not cached.  Nothing in the
+// array must start at zero (the pooling kernel writes every mean before the
+// logit kernel reads it), so no call clears it.  All calls on a device share
+// the one array: calls that overlap on the GPU (other streams, unordered host
 // threads) race on it.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -34,14 +41,48 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char velox_noalloc_scratch[kNoAllocScratchBytes];
 
 struct DeviceScratch {
-  std::once_flag once;
-  cudaError_t err = cudaErrorUnknown;
+  std::mutex mu;
+  bool valid = false;
+  unsigned long long ctx_id = 0;  // context the cached address belongs to
   void *ptr = nullptr;
 };
 DeviceScratch g_scratch[kMaxDevices];
 
-// Device address of the scratch array on the current device (set up once per
-// device); null with *err set when the lookup failed.
+// Driver entry points for the current context and its id (CUDA 12.0+).
+struct CtxFns {
+  PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  PFN_cuCtxGetId_v12000 get_id = nullptr;
+};
+const CtxFns &ctx_fns() {
+  static CtxFns f;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    cudaGetLastError();
+  });
+  return f;
+}
+
+// Id of the calling thread's current context; false when there is none yet.
+bool current_ctx_id(unsigned long long *id) {
+  const CtxFns &f = ctx_fns();
+  if (!f.get_current || !f.get_id) return false;
+  CUcontext ctx = nullptr;
+  if (f.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return f.get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array on the current device, looked up on
+// the first call in the device's current context; null with *err set when
+// the lookup failed.
 void *scratch_on_current_device(cudaError_t *err) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -51,17 +92,26 @@ void *scratch_on_current_device(cudaError_t *err) {
     return nullptr;
   }
   DeviceScratch &s = g_scratch[dev];
-  std::call_once(s.once, [&s] {
-    void *p = nullptr;
-    s.err = cudaGetSymbolAddress(&p, velox_noalloc_scratch);
-    if (s.err == cudaSuccess) {
-      s.ptr = p;
-    } else {
-      cudaGetLastError();
-    }
-  });
-  *err = s.err;
-  return s.err == cudaSuccess ? s.ptr : nullptr;
+  std::lock_guard<std::mutex> lock(s.mu);
+  unsigned long long id = 0;
+  if (s.valid && current_ctx_id(&id) && id == s.ctx_id) {
+    *err = cudaSuccess;
+    return s.ptr;
+  }
+  void *p = nullptr;
+  e = cudaGetSymbolAddress(&p, velox_noalloc_scratch);  // creates the context if needed
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    s.valid = false;
+    *err = e;
+    return nullptr;
+  }
+  // cache only when the context can be named, so a later context is noticed
+  s.valid = current_ctx_id(&id);
+  s.ctx_id = id;
+  s.ptr = p;
+  *err = cudaSuccess;
+  return p;
 }
 
 }  // namespace

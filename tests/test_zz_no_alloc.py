@@ -18,7 +18,7 @@ import numpy as np
 import pytest
 import torch
 
-from parity import P_RTOL, f64
+from parity import P_RTOL, f64, oracle_importance
 from synth.configs import small
 from synth import config, make_inputs
 
@@ -44,9 +44,13 @@ def _no_alloc(rbs, inp):
 
 def test_no_alloc_matches_workspace_entry_on_consecutive_calls():
     import routed_block_sparse_b200 as rbs
-    # two calls in a row on different shapes: the second call inherits the
-    # first call's leftovers in the shared array and must not depend on them
-    cases = [make_inputs(config(2), "cuda"), make_inputs(small(3, 5, 301, 0), "cuda")]
+    # calls in a row on different shapes: each call inherits the previous
+    # call's leftovers in the shared array and must not depend on them.  The
+    # first case has N > 96 query blocks, so its key means go through the
+    # array (the unfused path) and the fused calls after it find key means
+    # left behind there.
+    cases = [make_inputs(small(2, 100, 300, 0), "cuda"), make_inputs(config(2), "cuda"),
+             make_inputs(small(3, 5, 301, 0), "cuda")]
     for inp in cases:
         ref = _with_workspace(rbs, inp)
         got = _no_alloc(rbs, inp)
@@ -54,6 +58,10 @@ def test_no_alloc_matches_workspace_entry_on_consecutive_calls():
         g, r = f64(got), f64(ref)
         assert np.all(np.isfinite(g))
         assert np.all(np.abs(g - r) <= P_RTOL * np.abs(r)), "no-alloc importance differs"
+        # and against the oracle's definition, on up to three heads
+        heads = range(min(3, inp.wl.heads))
+        for h, ph in oracle_importance(inp.Q, inp.K, heads, 1.0).items():
+            assert np.abs(g[h] / ph - 1.0).max() <= P_RTOL, f"head {h} vs oracle"
 
 
 def test_no_alloc_rejects_sizes_beyond_its_array():
