@@ -22,7 +22,9 @@ Tolerances (written out here, derived in the design notes):
   touches have the same hole pattern and depths within MW_RTOL (the GPU's
   fp32 projection against fp64: a few ulps of coordinates of size ~10 after
   a 3x cancellation, ~2e-6 relative).  Every test counts its marginal cases
-  and bounds them by MARGINAL_FRAC of the pairs or tokens.
+  and bounds them by MARGINAL_FRAC of the pairs or tokens (at least 2): the
+  bound keeps the oracle from passing a test by calling everything
+  marginal; the values themselves are held to the ranges above.
 * attention O: bf16 inputs, fp32 accumulation, bf16 P and bf16 output:
   max |O_gpu - O_ref| <= 2e-2 and sum |O_gpu - O_ref| / sum |O_ref| <= 5e-3;
   lse within LSE_ATOL.
@@ -44,7 +46,10 @@ O_MEAN_REL = 5e-3
 LSE_ATOL = 1e-3
 G_RTOL = 4e-6
 MW_RTOL = 1e-5
-MARGINAL_FRAC = 0.01
+MARGINAL_FRAC = 0.05
+# a marginal sample marks up to 4 candidate tokens, and a small frame takes
+# s^2 samples per token from every source: a looser guard for multiwarp
+UNSURE_FRAC = 0.15
 
 
 def f64(t: torch.Tensor) -> np.ndarray:
@@ -149,7 +154,7 @@ def check_g_bounds(g_gpu, g, g_lo, g_hi):
     assert np.all(g_gpu[m] >= g_lo[m] * (1 - G_RTOL)), "g below the marginal range"
     assert np.all(g_gpu[m] <= g_hi[m] * (1 + G_RTOL)), "g above the marginal range"
     n_marg = int(m.sum())
-    assert n_marg <= MARGINAL_FRAC * g.size, f"{n_marg} marginal pairs"
+    assert n_marg <= max(2, MARGINAL_FRAC * g.size), f"{n_marg} marginal pairs"
     return n_marg
 
 
@@ -164,7 +169,7 @@ def check_coverage_bounds(rho_gpu, cov_gpu, n, n_lo, n_hi, b, eta):
     assert np.array_equal(cnt[fixed], n[fixed]), "covered count differs where it is fixed"
     assert np.array_equal(cov_gpu, (rho_gpu >= np.float32(eta)).astype(np.uint8))
     n_marg = int((~fixed).sum())
-    assert n_marg <= max(1, MARGINAL_FRAC * len(n) * b), f"{n_marg} marginal blocks"
+    assert n_marg <= max(2, MARGINAL_FRAC * len(n)), f"{n_marg} marginal blocks"
     return n_marg
 
 
@@ -175,5 +180,5 @@ def check_multiwarp(zq_gpu, zq_ref, unsure):
     nz = sure & (zq_ref != 0)
     assert np.all(np.abs(zq_gpu[nz].astype(np.float64) / zq_ref[nz] - 1.0) <= MW_RTOL)
     n_uns = int(unsure.sum())
-    assert n_uns <= MARGINAL_FRAC * unsure.size, f"{n_uns} unsure tokens"
+    assert n_uns <= max(2, UNSURE_FRAC * unsure.size), f"{n_uns} unsure tokens"
     return n_uns
