@@ -49,61 +49,113 @@ def _peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+    """SM clock and clock-event reasons sampled while the timed region runs.
 
+    Reads only (NVML queries of the launching device, every `period_s`; the
+    nvidia-smi command line at 20 ms when NVML cannot be used).  __enter__
+    returns once the first sample has arrived, so a short timed region still
+    gets samples from its start.
+    """
+
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, device, period_s: float = 0.005):
+        self.device = torch.device(device)
+        self.period = period_s
+        self.samples = []      # (sm_mhz, set of reason names)
+        self.sm_max = None
+        self.source = None
+        self._stop = threading.Event()
         self._t = None
+        self.proc = None
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self._t = threading.Thread(target=self._read, daemon=True)
-            self._t.start()
+            self._start_nvml()
         except Exception:
-            self.proc = None
+            self._start_smi()
+        t0 = time.time()
+        while not self.samples and time.time() - t0 < 3.0 and (self._t and self._t.is_alive()):
+            time.sleep(0.002)
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _start_nvml(self):
+        import pynvml
+        pynvml.nvmlInit()
+        idx = torch.cuda._get_nvml_device_index(self.device)
+        h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+        self.sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+        reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        self.source = f"nvml (device {idx}, every {self.period * 1e3:.0f} ms)"
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    mhz = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                    r = int(reasons_fn(h))
+                    self.samples.append((mhz, {n for n, b in bits.items() if r & b}))
+                except Exception:
+                    pass
+                self._stop.wait(self.period)
+
+        self._t = threading.Thread(target=run, daemon=True)
+        self._t.start()
+
+    def _start_smi(self):
+        gpu = self.device.index or 0
+        try:
+            gpu = torch.cuda._get_nvml_device_index(self.device)
+        except Exception:
+            pass
+        self.proc = subprocess.Popen(
+            ["nvidia-smi", f"--id={gpu}", f"--query-gpu={self.QUERY}",
+             "--format=csv,noheader,nounits", "-lms", "20"],
+            stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        self.source = "nvidia-smi (every 20 ms)"
+
+        def run():
+            for line in self.proc.stdout:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    mhz = float(parts[1])
+                    self.sm_max = float(parts[2])
+                except ValueError:
+                    continue
+                self.samples.append((mhz, {n for n, v in zip(self.NAMES, parts[5:9])
+                                           if v.lower() == "active"}))
+
+        self._t = threading.Thread(target=run, daemon=True)
+        self._t.start()
 
     def __exit__(self, *exc):
+        self._stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
-            if self._t:
-                self._t.join(timeout=2)
+        if self._t:
+            self._t.join(timeout=2)
 
     def summary(self):
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [m for m, _ in self.samples]
+        reasons = set()
+        for _, r in self.samples:
+            reasons |= r
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.sm_max,
+                "sm_mhz_min": min(sm) if sm else None, "reasons": sorted(reasons),
+                "samples": len(sm), "source": self.source}
 
 
 def _dist_setup():
@@ -141,16 +193,43 @@ def _sum_over_ranks(x: float, world: int, device="cuda") -> float:
     return float(t.item())
 
 
-def rank_workload(rank: int, heads: int = 0):
-    """Weak scaling: rank r runs layer r of the chunk-48 workload (its own
-    seeds); the path has no exchange between ranks."""
+def head_range(rank: int, world: int, H: int):
+    """Heads [h0, h1) that rank `rank` of `world` owns when the H heads of one
+    layer are split across ranks: contiguous, sizes differing by at most one,
+    every head owned by exactly one rank."""
+    return rank * H // world, (rank + 1) * H // world
+
+
+def rank_workload(rank: int, world: int = 1, heads: int = 0, shard: str = "heads"):
+    """The chunk-48 layer share of one rank, and its heads within the layer.
+
+    shard="heads" (default): rank r runs heads head_range(r, world, 40) of
+    layer 0 -- one layer split across the ranks (strong scaling).  Heads are
+    independent in every step of the path and g, the coverage flags and the
+    neighbour table are shared inputs, so no data crosses between ranks.
+    shard="layers": rank r runs all heads of its own layer r (weak scaling).
+    `heads` > 0 reduces the head count (profiler captures only, never a
+    bench value).
+    """
+    from dataclasses import replace
     from synth import config
-    wl = config(3, layer=rank)
+    wl = config(3, layer=rank if shard == "layers" else 0)
     if heads:
-        # reduced head count: only for small profiler captures, never a bench value
-        from dataclasses import replace
         wl = replace(wl, heads=heads)
-    return wl
+    if shard == "layers" or world == 1:
+        return wl, (0, wl.heads)
+    return wl, head_range(rank, world, wl.heads)
+
+
+def bench_config(wl, heads=None) -> dict:
+    """The `config` object of the bench line (both arms)."""
+    T, Hl, Wl = wl.lattice
+    H = wl.heads
+    return {"workload": "chunk48" if H == 40 else f"chunk48 reduced to {H} heads",
+            "heads": H, "n_q_blocks": wl.n_q_blocks, "n_kv_blocks": wl.n_kv_blocks,
+            "head_dim": wl.d, "b_tok": wl.b, "k_cov": wl.params.k_cov,
+            "k_unc": wl.params.k_unc, "theta": wl.params.theta_unc, "lattice": [T, Hl, Wl],
+            "l2": "inputs larger than L2 (K+V 5.9 GB per layer), no flush"}
 
 
 def aggregate(flops_step: float, ms_step: float, world: int, device="cuda"):
@@ -237,33 +316,75 @@ def cpu_oracle_sample(inp, attn_rows: int = 48, heads=tuple(range(12)), step_hea
 
 
 def run_reference(args, world, rank):
-    """--impl reference: the CPU oracle, on the host cores, rank 0 only."""
+    """--impl reference: the CPU oracle, as it stands, on the host cores.
+
+    Rank 0 only.  Each step is a bounded sample of the chunk-48 layer: one
+    whole head (1/40 of the layer's work) -- its importance over all 48 x
+    2256 blocks, the routes of its 48 query blocks and attention of those 48
+    rows -- timed as it runs; value = that head's routed-attention FLOPs over
+    the measured time, the same metric and unit as the GPU arm.  The Gilbert
+    neighbour table, built once per layer (about 0.2 % of the oracle's layer
+    time), is built once before the steps and reported on its own.
+    """
     if rank != 0:
         return
     import dataclasses
+    from oracle import attention as oatt
+    from oracle import gilbert as ogil
+    from oracle import importance as oimp
+    from oracle import route as ort
     from synth import config, make_inputs
+    from threadpoolctl import threadpool_info
+
     wl = config(3)
-    # the sample works on one head: draw a one-head layer of the same shape
-    # and distributions (drawing all 40 heads on the CPU would take minutes)
+    # one head of the chunk-48 shape and distributions (drawing all 40 heads
+    # on the CPU would take minutes)
     inp = make_inputs(dataclasses.replace(wl, heads=1), "cpu")
-    # FLOPs of the step: mean route length of the sampled head's oracle routes
-    times, flops_step = [], None
-    cache = {}
-    for s in range(args.warmup + args.steps):
-        r = cpu_oracle_sample(inp, attn_rows=8, heads=(0,), step_heads=wl.heads, cache=cache)
-        if s >= args.warmup:
-            times.append(r["step_s"])
-        if flops_step is None:
-            flops_step = 4.0 * 128 ** 3 * wl.heads * wl.n_q_blocks * r["mean_len"]
-    mean_s = sum(times) / len(times)
-    value = flops_step / mean_s / 1e12
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_s * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic",
-            "config": {"workload": "chunk48 (H=40, N=48, M=2256, d=128, b_tok=128)"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": r["threads"],
-                             "kind": "oracle", "sample": r["sample"]},
+    H, N, M, b = wl.heads, wl.n_q_blocks, wl.n_kv_blocks, wl.b
+    prm = ort.Params(lam=wl.params.lam, tau=wl.params.tau, g_ref=wl.params.g_ref,
+                     theta_cov=wl.params.theta_cov, theta_unc=wl.params.theta_unc,
+                     k_cov=wl.params.k_cov, k_unc=wl.params.k_unc)
+    Qh, Kh, Vh = (x[0].to(torch.float64).numpy() for x in (inp.Q, inp.K, inp.V))
+    g, cov = inp.g.numpy(), inp.covered.numpy()
+    T, Hl, Wl = wl.lattice
+    t0 = time.perf_counter()
+    nbr = ogil.neighbour_blocks(T, Hl, Wl, wl.n_chunks, b, wl.q_chunk, wl.cache_first_block, M)
+    t_nbr = time.perf_counter() - t0
+
+    def one_head():
+        p = oimp.importance(Qh, Kh, b, 1.0).astype(np.float32)
+        routes = [ort.route_row(p[i], g[i], bool(cov[i]), prm, wl.prev_begin, wl.prev_count,
+                                nbr[i]) for i in range(N)]
+        tiles = 0
+        for i in range(N):
+            ids = routes[i][0] + routes[i][1]
+            oatt.routed_attention_block(Qh[i * b:(i + 1) * b], Kh, Vh, ids, b)
+            tiles += len(ids)
+        return tiles
+
+    times, flops = [], []
+    for st in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        tiles = one_head()
+        dt = time.perf_counter() - t0
+        if st >= args.warmup:
+            times.append(dt)
+            flops.append(4.0 * b * b * wl.d * tiles)
+    value = sum(flops) / sum(times) / 1e12
+    threads = [x.get("num_threads", 1) for x in threadpool_info() if x.get("user_api") == "blas"]
+    cores = max(threads) if threads else 1
+    sample = (f"one whole head per step (1/{H} of the chunk-48 layer): importance ({N}x{M} "
+              f"blocks), routes of its {N} query blocks, attention of those {N} rows; "
+              f"fp64 numpy oracle, {cores} BLAS threads")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": max(world, args.gpus), "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": statistics.mean(times) * 1e3, "higher_is_better": True,
+            "scaling": "strong" if args.shard == "heads" else "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic (the GPU arm's recipe, one head)",
+            "config": bench_config(wl), "sample_per_step": sample,
+            "neighbour_table_ms": t_nbr * 1e3,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -276,8 +397,9 @@ def run_velox(args, world, rank, local):
     from synth import make_inputs
 
     dev = torch.device("cuda", local if world > 1 else 0)
-    wl = rank_workload(rank, args.heads)
-    inp = make_inputs(wl, dev)
+    wl_layer, (h0, h1) = rank_workload(rank, world, args.heads, args.shard)
+    inp = make_inputs(wl_layer, dev, heads=(h0, h1))
+    wl = inp.wl  # this rank's heads
     layer = layer_for(wl, device=dev)
     H, N, M, b, d = wl.heads, wl.n_q_blocks, wl.n_kv_blocks, wl.b, wl.d
     T, Hl, Wl = wl.lattice
@@ -314,7 +436,7 @@ def run_velox(args, world, rank, local):
     t_end = torch.cuda.Event(enable_timing=True)
     _barrier(world)
     torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index or 0) as clocks:
+    with ClockSampler(dev) as clocks:
         t_start.record(stream)
         for k in range(args.steps):
             step(evs[k])
@@ -350,30 +472,34 @@ def run_velox(args, world, rank, local):
         except Exception:
             traffic = None
 
+    clk = clocks.summary()
+    strong = args.shard == "heads"
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "strong" if strong else "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V; g U[0,1] half zeroed; coverage Bernoulli 0.5)",
-        "config": {"workload": "chunk48" if H == 40 else f"chunk48 reduced to {H} heads",
-                   "heads": H, "n_q_blocks": N, "n_kv_blocks": M,
-                   "head_dim": d, "b_tok": b, "k_cov": wl.params.k_cov, "k_unc": wl.params.k_unc,
-                   "theta": wl.params.theta_unc, "lattice": [T, Hl, Wl],
-                   "l2": "inputs larger than L2 (K+V 5.9 GB per layer), no flush"},
+        "config": bench_config(wl_layer),
+        "shard": ({"by": "heads", "heads_of_rank0": [h0, h1], "layer": 0} if strong and world > 1
+                  else {"by": args.shard if world > 1 else "none"}),
         "attn_us": attn_ms * 1e3, "attn_tflops": attn_tflops,
         "importance_us": imp_ms * 1e3, "importance_gbs": imp_gbs,
         "route_us": route_ms * 1e3, "gilbert_us": gil_ms * 1e3,
         "importance_route_gbs": ir_gbs, "importance_route_hbm_frac": ir_gbs / hbm,
         "routed_tiles": tiles, "mean_route_len": tiles / (H * N), "dev_status": status,
-        # the attention kernel is timed inside a ~1 s loop of back-to-back steps
-        # that runs under the 1 kW power cap (see "clocks"), so its denominator
-        # is the measured sustained bf16 figure; the burst fraction is reported too
-        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": bf16_sus,
-                     "unit": "TFLOP/s", "frac": attn_tflops / bf16_sus, "traffic": traffic,
-                     "peak_source": f"{peak_kind} bf16 dense, sustained under the power cap",
-                     "frac_of_burst_peak": attn_tflops / bf16, "burst_peak": bf16},
+        # the timed loop is short (tens to hundreds of ms), so the denominator
+        # is the measured burst bf16 figure; the sustained (power-capped)
+        # figure and the fraction against it are reported beside it, and the
+        # clock-normalised time (us x median SM MHz) lets runs on boxes that
+        # settle at different clocks be compared
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": bf16,
+                     "unit": "TFLOP/s", "frac": attn_tflops / bf16, "traffic": traffic,
+                     "peak_source": f"{peak_kind} bf16 dense burst (cuBLAS 8192^3, best of 10)",
+                     "sustained_peak": bf16_sus, "frac_of_sustained_peak": attn_tflops / bf16_sus,
+                     "attn_mcycles_per_call": (attn_ms * 1e3 * clk["sm_mhz"] / 1e6
+                                               if clk["sm_mhz"] else None)},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
-        "clocks": clocks.summary(),
+        "clocks": clk,
     }
 
     # the same step captured once as a CUDA graph and replayed (the seven
@@ -501,13 +627,13 @@ def _time_us(fn, reps=50, warm=3):
     return a.elapsed_time(b) / reps * 1e3
 
 
-def run_geometry(args):
-    """The geometry chain at the chunk-48 shape, one JSON line of per-call
-    times (not the bench line): slab table of the 2256 history blocks (188
-    frames of 32 x 48 tokens, 2 x 2 depth samples per token), multiwarp depth
-    of the 4 current frames from the first and last frames of the 30 most
-    recent chunks, the current chunk's 48 query slabs and tokens, slab
-    overlap g (8^3 samples per pair) and coverage rho."""
+def _geometry_chain(layout: str = "gilbert", seed: int = 20261203):
+    """The geometry chain at the chunk-48 shape for one token order: slab
+    table of the 2256 history blocks (188 frames of 32 x 48 tokens, 2 x 2
+    depth samples per token), multiwarp depth of the 4 current frames from the
+    first and last frames of the 30 most recent chunks, the current chunk's 48
+    query slabs and tokens, slab overlap g (8^3 samples per pair) and coverage
+    rho.  Returns the buffers and the five calls (not yet run)."""
     import numpy as np
     import routed_block_sparse_b200 as rbs
     from synth.depth import make_rollout
@@ -517,64 +643,130 @@ def run_geometry(args):
     per_chunk = T * H * W // b
     M, N = q_chunk * per_chunk, per_chunk
     hist_frames = q_chunk * T
-    roll = make_rollout(20261203, nc * T, H, W, s)
+    roll = make_rollout(seed, nc * T, H, W, s)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     cams = dev(roll.cams)
     n_cam = cams.shape[0]
     depth, conf, mask = dev(roll.depth[:hist_frames]), dev(roll.conf[:hist_frames]), \
         dev(roll.mask[:hist_frames])
     cell = torch.empty(nc * T * H * W, dtype=torch.int32, device="cuda")
-    rbs.velox_gilbert_order(T, H, W, nc, b, cell_of_rank=cell)
+    order = rbs.velox_gilbert_order if layout == "gilbert" else rbs.velox_thw_linear_order
+    order(T, H, W, nc, b, cell_of_rank=cell)
     src = []
     for c in range(q_chunk - 1, q_chunk - 31, -1):          # 30 most recent chunks
         src += [c * T + T - 1, c * T]                        # last, first frame
     src_depth = dev(roll.depth[src])
     src_cam = torch.tensor(src, dtype=torch.int32, device="cuda")
     tgt_cam = torch.arange(hist_frames, hist_frames + T, dtype=torch.int32, device="cuda")
-    hs = torch.empty(M, 8, dtype=torch.int32, device="cuda")
-    qs = torch.empty(N, 8, dtype=torch.int32, device="cuda")
-    zq = torch.empty(T, H, W, device="cuda")
-    uvz = torch.empty(N, b, 3, device="cuda")
-    g = torch.empty(N, M, device="cuda")
-    rho = torch.empty(N, device="cuda")
-    cov = torch.empty(N, dtype=torch.uint8, device="cuda")
-    st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    mw_ws = torch.empty(rbs.velox_multiwarp_workspace_size(len(src), T, H, W), dtype=torch.uint8,
-                        device="cuda")
+    buf = {"hs": torch.empty(M, 8, dtype=torch.int32, device="cuda"),
+           "qs": torch.empty(N, 8, dtype=torch.int32, device="cuda"),
+           "zq": torch.empty(T, H, W, device="cuda"),
+           "uvz": torch.empty(N, b, 3, device="cuda"),
+           "g": torch.empty(N, M, device="cuda"),
+           "rho": torch.empty(N, device="cuda"),
+           "cov": torch.empty(N, dtype=torch.uint8, device="cuda"),
+           "st": torch.zeros(1, dtype=torch.int32, device="cuda"),
+           "mw_ws": torch.empty(rbs.velox_multiwarp_workspace_size(len(src), T, H, W),
+                                dtype=torch.uint8, device="cuda")}
+    B = buf
 
     def table():
         rbs.velox_slab_table(depth, conf, mask, hist_frames, 0, H, W, s, cell, cell.numel(), b, 0,
-                             M, 0.5, 16, 0.1, 0.9, hs, st)
+                             M, 0.5, 16, 0.1, 0.9, B["hs"], B["st"])
 
     def warp():
-        rbs.velox_multiwarp(cams, n_cam, src_depth, src_cam, len(src), tgt_cam, T, H, W, s, 2, zq,
-                            mw_ws, st)
+        rbs.velox_multiwarp(cams, n_cam, src_depth, src_cam, len(src), tgt_cam, T, H, W, s, 2,
+                            B["zq"], B["mw_ws"], B["st"])
 
     def qtable():
-        rbs.velox_slab_table(zq, None, None, T, hist_frames, H, W, 1, cell, cell.numel(), b,
-                             q_chunk * per_chunk, N, 0.5, 8, 0.1, 0.9, qs, st, token_uvz=uvz)
+        rbs.velox_slab_table(B["zq"], None, None, T, hist_frames, H, W, 1, cell, cell.numel(), b,
+                             q_chunk * per_chunk, N, 0.5, 8, 0.1, 0.9, B["qs"], B["st"],
+                             token_uvz=B["uvz"])
 
     def overlap():
-        rbs.velox_slab_overlap(cams, n_cam, qs, N, hs, M, 8, g, st)
+        rbs.velox_slab_overlap(cams, n_cam, B["qs"], N, B["hs"], M, 8, B["g"], B["st"])
 
     def coverage():
-        rbs.velox_coverage(cams, n_cam, qs, uvz, N, b, hs, M, 0.9, rho, cov, st)
+        rbs.velox_coverage(cams, n_cam, B["qs"], B["uvz"], N, b, B["hs"], M, 0.9, B["rho"],
+                           B["cov"], B["st"])
 
-    out = {"geometry": "chunk48", "N": N, "M": M, "grid": 8, "b": b, "depth_samples": s,
-           "multiwarp_sources": len(src)}
-    for name, fn in (("slab_table", table), ("multiwarp", warp), ("query_slabs", qtable),
-                     ("slab_overlap", overlap), ("coverage", coverage)):
+    calls = (("slab_table", table), ("multiwarp", warp), ("query_slabs", qtable),
+             ("slab_overlap", overlap), ("coverage", coverage))
+    meta = {"N": N, "M": M, "grid": 8, "b": b, "depth_samples": s,
+            "multiwarp_sources": len(src)}
+    return buf, calls, meta
+
+
+def run_geometry(args):
+    """The geometry chain at the chunk-48 shape (Gilbert order), one JSON
+    line of per-call times (not the bench line)."""
+    buf, calls, meta = _geometry_chain("gilbert")
+    out = {"geometry": "chunk48", **meta}
+    for name, fn in calls:
         out[name + "_us"] = _time_us(fn)
 
     def chain():
-        table(); warp(); qtable(); overlap(); coverage()
+        for _, fn in calls:
+            fn()
     out["chain_us"] = _time_us(chain, reps=20)
     torch.cuda.synchronize()
-    out.update({"valid_history_slabs": int(hs[:, 7].sum().item()),
-                "query_holes": float((zq == 0).float().mean().item()),
-                "nonzero_pairs": int((g > 0).sum().item()),
-                "covered_blocks": int(cov.sum().item()), "dev_status": int(st.item())})
+    out.update({"valid_history_slabs": int(buf["hs"][:, 7].sum().item()),
+                "query_holes": float((buf["zq"] == 0).float().mean().item()),
+                "nonzero_pairs": int((buf["g"] > 0).sum().item()),
+                "covered_blocks": int(buf["cov"].sum().item()),
+                "dev_status": int(buf["st"].item())})
     print(json.dumps(out), flush=True)
+
+
+def _route_runs(route_ids: torch.Tensor, route_len: torch.Tensor):
+    """Mean route length and mean length of the runs of consecutive block
+    ids in the routes (each route taken as a sorted set)."""
+    ids = route_ids.cpu().numpy().reshape(-1, route_ids.shape[-1])
+    lens = route_len.cpu().numpy().reshape(-1)
+    total = runs = 0
+    for r in range(ids.shape[0]):
+        v = np.sort(ids[r, :lens[r]])
+        if len(v):
+            total += len(v)
+            runs += 1 + int(np.count_nonzero(np.diff(v) != 1))
+    return total / max(1, ids.shape[0]), total / max(1, runs)
+
+
+def run_layouts(args):
+    """Gilbert against THW-linear token order through the whole routed path
+    at the chunk-48 shape: the geometry chain of each order (slab tables from
+    the same depth maps, multiwarp, g, coverage), then importance, route
+    build and attention on the same Q/K/V.  One JSON line per order: mean
+    route length, mean run of consecutive block ids in a route, attention
+    time.  `--layout` restricts it to one order (for an ncu capture)."""
+    from routed_block_sparse_b200.pipeline import layer_for
+    from synth import config, make_inputs
+
+    wl = config(3)
+    if args.heads:
+        from dataclasses import replace
+        wl = replace(wl, heads=args.heads)
+    inp = make_inputs(wl, "cuda")
+    for layout in (("gilbert", "thw") if args.layout == "both" else (args.layout,)):
+        buf, calls, _ = _geometry_chain(layout)
+        for _, fn in calls:
+            fn()
+        layer = layer_for(wl, order=layout)
+        layer.importance(inp.Q, inp.K)
+        layer.route(buf["g"], buf["cov"])
+        torch.cuda.synchronize()
+        mean_len, mean_run = _route_runs(layer.route_ids, layer.route_len)
+        t_att = _time_us(lambda: layer.attend(inp.Q, inp.K, inp.V), reps=20)
+        tiles = float(layer.route_len.sum().item())
+        print(json.dumps({"layout": layout, "config": bench_config(wl),
+                          "g_nonzero_pairs": int((buf["g"] > 0).sum().item()),
+                          "covered_blocks": int(buf["cov"].sum().item()),
+                          "mean_route_len": mean_len, "mean_run_len": mean_run,
+                          "attn_us": t_att,
+                          "attn_tflops": 4.0 * 128 ** 3 * tiles / (t_att * 1e-6) / 1e12,
+                          "dev_status": layer.status() | int(buf["st"].item())}), flush=True)
+        del layer, buf
+        torch.cuda.empty_cache()
 
 
 def run_two_phase(args):
@@ -716,11 +908,25 @@ def _attn_source_hash() -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
+def _spawn_ranks(n: int) -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__),
+           *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--shard", default="heads", choices=["heads", "layers"],
+                    help="N > 1: split one layer's heads over the ranks (strong scaling) or "
+                         "give every rank its own layer (weak scaling)")
     ap.add_argument("--impl", default="velox", choices=["velox", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -735,11 +941,17 @@ def main():
     ap.add_argument("--layers", type=int, default=0,
                     help="full-step mode: this many chunk-48 layers with per-layer inputs "
                          "(extra line with the summed route-build and attention times)")
+    ap.add_argument("--layouts", action="store_true",
+                    help="Gilbert vs THW-linear order through geometry, routes and attention")
+    ap.add_argument("--layout", default="both", choices=["both", "gilbert", "thw"])
     ap.add_argument("--heads", type=int, default=0,
                     help="run a reduced head count (profiler captures only)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ and args.impl == "velox":
+        # start one rank per GPU (the same command under torch.distributed.run)
+        sys.exit(_spawn_ranks(args.gpus))
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -752,6 +964,9 @@ def main():
             return
         if args.geometry:
             run_geometry(args)
+            return
+        if args.layouts:
+            run_layouts(args)
             return
         if args.variants:
             run_variants(args)

@@ -24,7 +24,7 @@ import torch
 
 from . import (BLOCK_TOK, HEAD_DIM, RouteParams, route_params, velox_block_importance,
                velox_block_sparse_attn, velox_gilbert_order, velox_route_build,
-               velox_route_schedule, velox_workspace_size)
+               velox_route_schedule, velox_thw_linear_order, velox_workspace_size)
 
 DEFAULT_S_MAX = 64
 
@@ -34,7 +34,7 @@ class RoutedLayer:
                  prev_begin: int = 0, prev_count: int = 0, lattice=None, q_chunk: int = 0,
                  cache_first_block: int = 0, S_max: int = DEFAULT_S_MAX,
                  ref_ids: Optional[torch.Tensor] = None, importance_scale: float = 1.0,
-                 softmax_scale: float = 0.0, device="cuda"):
+                 softmax_scale: float = 0.0, order: str = "gilbert", device="cuda"):
         self.H, self.N, self.M = H, N, M
         self.b, self.d = BLOCK_TOK, HEAD_DIM
         self.prm = prm if prm is not None else route_params()
@@ -56,9 +56,15 @@ class RoutedLayer:
             self.S_max = S_max
             self.nbr_ids = torch.empty(N, S_max, dtype=i32, device=dev)
             self.nbr_cnt = torch.empty(N, dtype=i32, device=dev)
-            velox_gilbert_order(T, Hl, Wl, n_chunks, self.b, q_chunk, cache_first_block, M,
-                                nbr_ids=self.nbr_ids, nbr_cnt=self.nbr_cnt, S_max=S_max,
-                                dev_status=self.dev_status)
+            # the neighbour table of the token order the cache is stored in:
+            # the global Gilbert order, or the THW-linear (raster) order the
+            # pages compare it with
+            if order not in ("gilbert", "thw"):
+                raise ValueError(f"unknown order {order!r}")
+            fn = velox_gilbert_order if order == "gilbert" else velox_thw_linear_order
+            fn(T, Hl, Wl, n_chunks, self.b, q_chunk, cache_first_block, M,
+               nbr_ids=self.nbr_ids, nbr_cnt=self.nbr_cnt, S_max=S_max,
+               dev_status=self.dev_status)
         else:
             self.S_max = 0
             self.nbr_ids = self.nbr_cnt = None

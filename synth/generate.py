@@ -60,8 +60,24 @@ def _geometry(wl: Workload):
     return g.contiguous(), covered.contiguous()
 
 
-def make_inputs(wl: Workload, device="cpu", out: Optional[Inputs] = None) -> Inputs:
-    """Draw the inputs of ``wl`` on ``device``; reuse ``out``'s buffers if given."""
+def make_inputs(wl: Workload, device="cpu", out: Optional[Inputs] = None,
+                heads: Optional[tuple] = None) -> Inputs:
+    """Draw the inputs of ``wl`` on ``device``; reuse ``out``'s buffers if given.
+
+    ``heads=(h0, h1)`` keeps only heads h0..h1-1 of Q, K and V: the values are
+    those heads of the full draw (the whole layer is drawn, then cut), so the
+    shares of several ranks put together are the single-rank inputs.  The
+    returned workload then has h1 - h0 heads.
+    """
+    if heads is not None:
+        from dataclasses import replace
+        h0, h1 = heads
+        if not (0 <= h0 < h1 <= wl.heads):
+            raise ValueError(f"head range {heads} outside 0..{wl.heads}")
+        full = make_inputs(wl, device)
+        cut = lambda t: t[h0:h1].clone()
+        return Inputs(wl=replace(wl, heads=h1 - h0), Q=cut(full.Q), K=cut(full.K),
+                      V=cut(full.V), g=full.g, covered=full.covered, ref_ids=full.ref_ids)
     device = torch.device(device)
     H, N, M, b, d = wl.heads, wl.n_q_blocks, wl.n_kv_blocks, wl.b, wl.d
     gen = torch.Generator(device=device).manual_seed(wl.seed)

@@ -91,15 +91,81 @@ def test_pipeline_sweep_and_dense(lib):
         torch.cuda.empty_cache()
 
 
+def _routes_from_gpu_p(layer, inp, nbr):
+    """Oracle routes of every (head, query block) row from the GPU's own p
+    (the route step's input), compared with the GPU routes: bit-exact except
+    at a mass cut within MASS_EPS of theta.  Returns {(h, i): tile list}."""
+    from oracle import route as ort
+    from parity import check_route_row
+    wl = inp.wl
+    prm = oracle_params(wl.params)
+    p = layer.p.cpu().numpy()
+    g, cov = inp.g.cpu().numpy(), inp.covered.cpu().numpy()
+    rid, rlen, rnb = layer.route_ids.cpu(), layer.route_len.cpu(), layer.route_nbudget.cpu()
+    out, n_cut = {}, 0
+    for h in range(wl.heads):
+        for i in range(wl.n_q_blocks):
+            ref = ort.route_row(p[h, i], g[i], bool(cov[i]), prm, wl.prev_begin,
+                                wl.prev_count, list(nbr[i]))
+            gpu = gpu_row(rid, rlen, rnb, h, i)
+            n_cut += check_route_row(gpu, ref, f"head {h} row {i}") == "cut"
+            out[(h, i)] = gpu[0] + gpu[1]
+    return out, n_cut
+
+
 @pytest.mark.slow
-def test_pipeline_forty_layers_routes(lib):
-    # the 40-layer workload: per-layer seeds into reused buffers; routes of two layers and
-    # attention rows of one checked (the oracle is the slow side)
+def test_pipeline_forty_layers(lib):
+    """The 40-layer workload (per-layer seeds, regenerated into reused
+    buffers): route sets of every head and query block of all 40 layers,
+    importance on 4 heads of every layer, attention on 4 heads x 8 rows of
+    layers 0 and 39."""
     wl0 = config(5, 0)
     layer = layer_for(wl0)
     inp = make_inputs(wl0, "cuda")
-    for layer_idx in (0, 39):
-        wl = config(5, layer_idx)
+    T, Hl, Wl = wl0.lattice
+    nbr = gilbert.neighbour_blocks(T, Hl, Wl, wl0.n_chunks, 128, wl0.q_chunk,
+                                   wl0.cache_first_block, wl0.n_kv_blocks)
+    from parity import P_RTOL
+    for li in range(40):
+        wl = config(5, li)
         inp = make_inputs(wl, "cuda", out=inp)
         layer.forward(inp.Q, inp.K, inp.V, inp.g, inp.covered)
-        _compare(layer, inp, [layer_idx % 40], (2,))
+        torch.cuda.synchronize()
+        assert layer.status() == 0, f"layer {li}"
+        routes, n_cut = _routes_from_gpu_p(layer, inp, nbr)
+        assert n_cut <= 2, f"layer {li}: {n_cut} rows differ at the cut"
+        heads = [(li + 10 * k) % 40 for k in range(4)]
+        for h, ph in oracle_importance(inp.Q, inp.K, heads).items():
+            rel = np.abs(f64(layer.p[h]) / ph - 1.0).max()
+            assert rel <= P_RTOL, f"layer {li} head {h}: importance rel err {rel}"
+        if li in (0, 39):
+            rng = np.random.default_rng(li)
+            rows = [(h, int(i)) for h in heads for i in rng.choice(48, size=8, replace=False)]
+            ref = attention_rows(inp.Q, inp.K, inp.V, rows, lambda h, i: routes[(h, i)])
+            assert_attention_close(layer.O, layer.lse, ref)
+
+
+@pytest.mark.slow
+def test_chunk48_attention_rows_of_every_wave(lib):
+    """The bench's launch (longest-route-first row order, one CTA per SM):
+    one row from each wave of that order, the last row of the final wave and
+    its neighbours, against the oracle on the layer's own routes."""
+    wl = config(3)
+    inp = make_inputs(wl, "cuda")
+    layer = layer_for(wl)
+    layer.forward(inp.Q, inp.K, inp.V, inp.g, inp.covered)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    order = layer.row_order.cpu().numpy()
+    lens = layer.route_len.cpu().numpy().reshape(-1)
+    assert np.all(np.diff(lens[order]) <= 0)       # longest first
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    rows_total = len(order)
+    pos = sorted(set(list(range(0, rows_total, sms)) + [rows_total - 3, rows_total - 2,
+                                                        rows_total - 1]))
+    N = wl.n_q_blocks
+    rows = sorted({(int(order[k]) // N, int(order[k]) % N) for k in pos})
+    rid, rlen = layer.route_ids.cpu(), layer.route_len.cpu()
+    routes = {(h, i): rid[h, i, :int(rlen[h, i])].tolist() for (h, i) in rows}
+    ref = attention_rows(inp.Q, inp.K, inp.V, rows, lambda h, i: routes[(h, i)])
+    assert_attention_close(layer.O, layer.lse, ref)
