@@ -922,7 +922,7 @@ def _spawn_ranks(n: int) -> int:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--shard", default="heads", choices=["heads", "layers"],
                     help="N > 1: split one layer's heads over the ranks (strong scaling) or "
