@@ -29,7 +29,7 @@
 // PV_j by the softmax threads of tile j.
 //   warpgroup 0 (56 registers per thread after setmaxnreg), one thread per
 //   warp active:
-//     warp 0    TMA producer of Q and of the route's K tiles, warp 2 of its V
+//     warp 0    TMA producer of the route's K tiles, warp 2 of its V
 //               tiles, into two rings of 32 KB slots (128-byte swizzle, two
 //               64-channel boxes per tile): a K slot is freed by its score
 //               product, a V slot by its PV, so neither stream waits on the
@@ -50,7 +50,7 @@
 //     in the reference of its own last tile; the epilogue brings both to the
 //     final reference and writes O / l and the lse.
 // A pre-pass compacts the route into shared memory, skipping ids outside
-// [0, M) and repeats (flagged in dev_status).
+// [0, M) and repeats (flagged in dev_status); Q's load is issued before it.
 //
 // Two-phase form (digest, "Reproducibility": the two-phase tile loop): after
 // the routed history tiles the same loop visits the n_cur tiles of the
@@ -102,10 +102,10 @@ constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffRing = kOffQ + kTileBytes;
 // barriers, misc, the reference hand-over and the route list follow the ring
 // (offsets set at launch).  Barriers: q_full, the K/V ring (full, empty),
-// per buffer s_full / s_free / p_full / pv_done / ref_full, x_fin, mma_done.
-constexpr uint32_t kNumBars = 1 + 2 * kMaxSlots + 5 * kBufs + 1 + 1;
+// per buffer s_full / s_free / p_full / pv_done, x_fin, mma_done.
+constexpr uint32_t kNumBars = 1 + 2 * kMaxSlots + 4 * kBufs + 1 + 1;
 constexpr uint32_t kMiscBytes = 64;
-constexpr uint32_t kRefBytes = BM * 4;  // one fp32 reference per row
+constexpr uint32_t kRefBytes = BM * 8;  // per row: reference bits, index of the tile that wrote it
 constexpr uint32_t kSmemLimit = 227 * 1024;
 
 struct AttnArgs {
@@ -154,6 +154,38 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
 }
 
+// The per-row reference word: {value bits, tile index}, stored and loaded
+// as one 64-bit shared-memory access so the pair is always consistent.
+__device__ __forceinline__ void ref_word_store(uint32_t saddr, uint32_t val, uint32_t tag) {
+  asm volatile("st.volatile.shared.v2.u32 [%0], {%1, %2};" ::"r"(saddr), "r"(val), "r"(tag)
+               : "memory");
+}
+// Polls the word until it carries `tag`; gives up (false, *abort set) after
+// the same time limit as mbar_wait, or when another thread has aborted.
+__device__ __forceinline__ bool ref_word_wait(uint32_t saddr, uint32_t tag, volatile int *abort,
+                                              float *val) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    uint32_t v, t;
+    asm volatile("ld.volatile.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v), "=r"(t) : "r"(saddr)
+                 : "memory");
+    if (t == tag) {
+      *val = __uint_as_float(v);
+      return true;
+    }
+    if ((it & 255u) == 255u) {
+      if (*abort) return false;
+      const uint64_t now = global_timer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // 2^x for a pair of fp32 values on the FMA pipe: x = k + f with k the
 // nearest integer (the 1.5 * 2^23 shifter puts k in the low mantissa bits)
 // and f in [-0.5, 0.5]; 2^f from a cubic fitted to it here by iterated
@@ -199,14 +231,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *s_free = s_full + kBufs;          // [buffer]: S_j read by its softmax
   uint64_t *p_full = s_free + kBufs;          // [buffer]: P_j written
   uint64_t *pv_done = p_full + kBufs;         // [buffer]: PV_j (and all before) done
-  uint64_t *ref_full = pv_done + kBufs;       // [buffer]: reference of tile j handed over
-  uint64_t *x_fin = ref_full + kBufs;         // both warpgroups' row sums written
+  uint64_t *x_fin = pv_done + kBufs;          // both warpgroups' row sums written
   uint64_t *mma_done = x_fin + 1;             // every MMA of the CTA done
   uint8_t *misc = base + a.bar_offset + kNumBars * 8;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(misc);
   int *s_nvalid = reinterpret_cast<int *>(misc + 4);
   volatile int *s_abort = reinterpret_cast<volatile int *>(misc + 8);
-  float *refx = reinterpret_cast<float *>(base + a.ref_offset);
+  uint32_t refx = smem_u32(base + a.ref_offset);  // [row] {reference bits, tile index}
   uint16_t *tiles = reinterpret_cast<uint16_t *>(base + a.list_offset);
   // the id bitmap of the route compaction lives in the ring, idle until the
   // first load
@@ -235,17 +266,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s_free[b], kChainThreads);
       mbar_init(&p_full[b], kChainThreads);
       mbar_init(&pv_done[b], 1);
-      mbar_init(&ref_full[b], kChainThreads);
     }
     mbar_init(x_fin, kSoftThreads);
     mbar_init(mma_done, 2);  // one commit from each MMA-issuing thread
     *s_abort = 0;
     fence_mbar_init();
+    // Q does not depend on the route: its load overlaps the compaction
+    prefetch_tmap(&tmQ);
+    mbar_arrive_expect_tx(q_full, kTileBytes);
+    tma_load_3d(sQ, &tmQ, q_full, 0, i * BM, h);
+    tma_load_3d(sQ + kHalfBytes, &tmQ, q_full, 64, i * BM, h);
   }
   if (warp == 1) {
     tmem_alloc(s_tmem, kTmemCols);
     tmem_relinquish();
   }
+  if (threadIdx.x < BM) ref_word_store(refx + threadIdx.x * 8, 0u, 0xFFFFFFFFu);  // no tile yet
   int L = 0;
   if (!dense) {
     L = a.route_len[row];
@@ -310,12 +346,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the ring held the compaction bitmap (generic-proxy writes) just
         // before these asynchronous copies overwrite it
         fence_proxy_async_smem();
-        if (is_k) {
-          prefetch_tmap(&tmQ);
-          mbar_arrive_expect_tx(q_full, kTileBytes);
-          tma_load_3d(sQ, &tmQ, q_full, 0, i * BM, h);
-          tma_load_3d(sQ + kHalfBytes, &tmQ, q_full, 64, i * BM, h);
-        }
         const int s0 = is_k ? 0 : kk;  // first slot of this ring
         int issued = 0;
         for (int j = 0; j < n; ++j) {
@@ -436,19 +466,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         mx[k & 7] = fmax3(mx[k & 7], __uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1]));
       const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
                              fmaxf(mx[6], mx[7])) * c;
-      // reference hand-over: tile j - 1 (the other warpgroup) wrote its
-      // reference to refx[r]; this tile raises it only on growth above 2^8
+      // reference hand-over: the thread of this row in the other warpgroup
+      // stores {reference, j - 1} as one 64-bit word once tile j - 1 has its
+      // max; this thread polls its own row's word (usually one load).  The
+      // word holds j - 2 or j - 1 when tile j reads it: tile j + 1 writes
+      // only after reading what tile j writes.  This tile raises the
+      // reference only on growth above 2^8.
       float ref_prev = -INFINITY;
       if (j > 0) {
-        if (!warp_wait(&ref_full[ch ^ 1], ((j - 1) >> 1) & 1, s_abort)) { ok = false; break; }
-        ref_prev = refx[r];
+        const bool got = ref_word_wait(refx + r * 8, (uint32_t)(j - 1), s_abort, &ref_prev);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       }
       const bool grow = mt > ref_prev + kRescaleThreshold;  // always on tile 0
       const float ref = grow ? mt : ref_prev;
-      if (j + 1 < n) {
-        refx[r] = ref;  // read by tile j + 1 only after this arrival
-        mbar_arrive(&ref_full[ch]);
-      }
+      if (j + 1 < n) ref_word_store(refx + r * 8, __float_as_uint(ref), (uint32_t)j);
       // P buffer reuse: PV_{j-2} (this buffer's last reader) must be done;
       // that also puts every PV before it behind us
       if (j >= 2 && !warp_wait(&pv_done[ch], ((j - 2) >> 1) & 1, s_abort)) { ok = false; break; }
@@ -557,6 +588,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           good ? (ref_fin + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
   }
 
+  if (threadIdx.x == 0 && n == 0) {
+    // nothing waited for Q: its copy must land before the CTA goes away
+    volatile int never = 0;
+    mbar_wait(q_full, 0, &never);
+  }
   if (*s_abort && threadIdx.x == 0) flag_error(a.dev_status, VELOX_DEV_WAIT_TIMEOUT);
   tc_fence_before();
   __syncthreads();
