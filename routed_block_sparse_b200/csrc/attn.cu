@@ -239,9 +239,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *s_abort = reinterpret_cast<volatile int *>(misc + 8);
   uint32_t refx = smem_u32(base + a.ref_offset);  // [row] {reference bits, tile index}
   uint16_t *tiles = reinterpret_cast<uint16_t *>(base + a.list_offset);
-  // the id bitmap of the route compaction lives in the ring, idle until the
-  // first load
+  // the id bitmap of the route compaction and the raw route live in the
+  // ring, idle until the first load (bitmap: M bits <= 8 KB; route: R_max
+  // int32 <= 16 KB after it)
   uint32_t *bits = reinterpret_cast<uint32_t *>(ring);
+  int32_t *raw = reinterpret_cast<int32_t *>(ring + 8192);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = a.row_order ? a.row_order[blockIdx.x] : (int)blockIdx.x;
@@ -291,18 +293,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const int W = (M + 31) >> 5;
     for (int k = threadIdx.x; k < W; k += kThreads) bits[k] = 0u;
+    // stage the route in shared memory in one parallel pass (one global
+    // round trip instead of one per 32 ids in the ordered pass below)
+    const int32_t *ids = a.route_ids + (size_t)row * a.R_max;
+    for (int k = threadIdx.x; k < L; k += kThreads) raw[k] = ids[k];
   }
   __syncthreads();
   if (warp == 0) {
     if (dense) {
       if (lane == 0) *s_nvalid = M;
     } else {
-      const int32_t *ids = a.route_ids + (size_t)row * a.R_max;
       int n = 0;
       bool bad = false, dup = false;
       for (int b0 = 0; b0 < L; b0 += 32) {
         const int j = b0 + lane;
-        const int id = j < L ? ids[j] : -1;
+        const int id = j < L ? raw[j] : -1;
         bool ok = (j < L) && id >= 0 && id < M;
         if (j < L && !ok) bad = true;
         if (ok) {
@@ -678,7 +683,9 @@ cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
   a.ref_offset = a.bar_offset + kNumBars * 8 + kMiscBytes;
   a.list_offset = a.ref_offset + kRefBytes;
   const size_t smem = (size_t)a.list_offset + list_bytes + 1024;  // + alignment slack
-  if (smem > kSmemLimit || (size_t)nslot * kTileBytes < (size_t)(M + 31) / 32 * 4)
+  // the compaction's bitmap (first 8 KB) and raw route (after it) fit in the ring
+  if (smem > kSmemLimit || (size_t)(M + 31) / 32 * 4 > 8192 ||
+      (size_t)nslot * kTileBytes < 8192 + (size_t)R_max * 4)
     return cudaErrorInvalidConfiguration;
   // The setmaxnreg split draws on the registers of the launch: refuse to
   // launch a build whose per-thread count is below the one it was planned for
