@@ -405,18 +405,30 @@ def run_velox(args, world, rank, local):
     T, Hl, Wl = wl.lattice
     stream = torch.cuda.current_stream(dev)
 
+    side = torch.cuda.Stream(dev)
+
+    # One step.  The neighbour table (a1) does not depend on the importance
+    # (a2, a3): it runs on a side stream forked at the start of the step and
+    # joined before the route build, which needs both.  Events: 0 step start,
+    # 1 / 2 importance start / end (main stream), 3 route end, 4 attention end,
+    # 5 / 6 neighbour table start / end (side stream).
     def step(ev=None, st=None):
         st = stream if st is None else st
         if ev is not None:
             ev[0].record(st)
+        side.wait_stream(st)
+        if ev is not None:
+            ev[5].record(side)
         rbs.velox_gilbert_order(T, Hl, Wl, wl.n_chunks, b, wl.q_chunk, wl.cache_first_block, M,
                                 nbr_ids=layer.nbr_ids, nbr_cnt=layer.nbr_cnt,
-                                S_max=layer.S_max, dev_status=layer.dev_status, stream=st)
+                                S_max=layer.S_max, dev_status=layer.dev_status, stream=side)
         if ev is not None:
+            ev[6].record(side)
             ev[1].record(st)
         layer.importance(inp.Q, inp.K, st)
         if ev is not None:
             ev[2].record(st)
+        st.wait_stream(side)
         layer.route(inp.g, inp.covered, stream=st)
         if ev is not None:
             ev[3].record(st)
@@ -431,7 +443,7 @@ def run_velox(args, world, rank, local):
     route_len = layer.route_len.to(torch.float64)
     tiles = float(route_len.sum().item())
     flops_step = 4.0 * b * b * d * tiles
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     _barrier(world)
@@ -445,7 +457,8 @@ def run_velox(args, world, rank, local):
     _barrier(world)
     torch.cuda.synchronize(dev)
     total_ms = t_start.elapsed_time(t_end)
-    parts = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])
+    parts = np.array([[e[5].elapsed_time(e[6]), e[1].elapsed_time(e[2]),
+                       e[2].elapsed_time(e[3]), e[3].elapsed_time(e[4])] for e in evs])
     gil_ms, imp_ms, route_ms, attn_ms = parts.mean(axis=0)
     value, ms_step = aggregate(flops_step, total_ms / args.steps, world)
 

@@ -92,6 +92,33 @@ def test_route_chunk48(lib):
     assert kinds["cut"] <= 2
 
 
+@pytest.mark.slow
+def test_route_chunk48_live_safeguards(lib):
+    """The chunk-48 layer with only the last 6 blocks reserved: the 26-
+    neighbour blocks of the query blocks in the chunk's first frame (blocks
+    2244-2255, the last frame of the previous chunk) are then mostly outside
+    the reserved set, so the safeguard append is live.  All 40 heads, GPU p
+    fed to both sides; route ids bit-exact."""
+    from routed_block_sparse_b200.pipeline import layer_for
+    wl = config(3)
+    inp = make_inputs(wl, "cuda")
+    layer = layer_for(wl)
+    p32 = layer.importance(inp.Q, inp.K).cpu().numpy()
+    T, Hl, Wl = wl.lattice
+    M = wl.n_kv_blocks
+    nbr = gilbert.neighbour_blocks(T, Hl, Wl, wl.n_chunks, 128, wl.q_chunk,
+                                   wl.cache_first_block, M)
+    g, cov = inp.g.cpu().numpy(), inp.covered.cpu().numpy()
+    kinds = _run_case(p32, g, cov, _prm(wl), M - 6, 6, nbr=nbr)
+    assert kinds["cut"] <= 2
+    # the extras really are appended: the query blocks of the chunk's first
+    # frame border the previous chunk's last frame and gain safeguards
+    oprm = oracle_params(_prm(wl))
+    ref = oracle_routes({0: p32[0]}, g, cov, oprm, M - 6, 6, nbr)
+    n_extra = [len(v[1]) for v in ref.values()]
+    assert sum(x > 0 for x in n_extra) >= 6 and max(n_extra) >= 4
+
+
 def _synthetic_p(H, N, M, seed, peaked=1.0, flat=False):
     r = np.random.default_rng(seed)
     if flat:
