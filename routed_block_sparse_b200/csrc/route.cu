@@ -24,6 +24,9 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+// up to this many candidates are ordered by a rank sort (O(k^2 / threads)
+// compares); more by a bitonic network in shared memory (O(k log^2 k))
+constexpr int kRankSortMax = 256;
 
 struct RouteArgs {
   const float *p;
@@ -41,7 +44,8 @@ struct RouteArgs {
   int32_t *route_ids, *route_len, *route_nbudget;
   int R_max;
   double *ws_keys;  // [rows][M] when the keys do not fit in shared memory
-  int kcap;         // candidate capacity = max(k_cov, k_unc) (>= 1)
+  int kcap;         // candidate capacity = max(k_cov, k_unc) (>= 1), rounded up to a
+                    // power of two when above kRankSortMax (the bitonic sort's length)
   int32_t *dev_status;
 };
 
@@ -254,17 +258,52 @@ __global__ void __launch_bounds__(kThreads) route_kernel(RouteArgs a) {
   }
   __syncthreads();
 
-  // ---- 3. rank sort (weight desc; candidates are in id order, so equal
-  //         weights keep ascending ids)
-  for (int x = tid; x < k_sel; x += kThreads) {
-    const double kx = cand_key[x];
-    int rank = 0;
-    for (int y = 0; y < k_sel; ++y) {
-      const double ky = cand_key[y];
-      rank += (ky > kx) || (ky == kx && y < x);
+  // ---- 3. sort the candidates: weight descending, ties to the lower id
+  //         (candidates arrive in id order)
+  if (k_sel <= kRankSortMax) {
+    for (int x = tid; x < k_sel; x += kThreads) {
+      const double kx = cand_key[x];
+      int rank = 0;
+      for (int y = 0; y < k_sel; ++y) {
+        const double ky = cand_key[y];
+        rank += (ky > kx) || (ky == kx && y < x);
+      }
+      sort_id[rank] = cand_id[x];
+      sort_s[rank] = cov ? (invZ_ok != 0.0 ? __ddiv_rn(kx, Z) : 0.0) : kx;
     }
-    sort_id[rank] = cand_id[x];
-    sort_s[rank] = cov ? (invZ_ok != 0.0 ? __ddiv_rn(kx, Z) : 0.0) : kx;
+  } else {
+    // bitonic network over the next power of two; padding (-1, INT_MAX)
+    // sorts after every weight (weights are >= 0)
+    int P = 1;
+    while (P < k_sel) P <<= 1;
+    for (int x = k_sel + tid; x < P; x += kThreads) {
+      cand_key[x] = -1.0;
+      cand_id[x] = 0x7FFFFFFF;
+    }
+    __syncthreads();
+    for (int k = 2; k <= P; k <<= 1) {
+      for (int jj = k >> 1; jj > 0; jj >>= 1) {
+        for (int x = tid; x < P; x += kThreads) {
+          const int y = x ^ jj;
+          if (y > x) {
+            const double kx = cand_key[x], ky = cand_key[y];
+            const int ix = cand_id[x], iy = cand_id[y];
+            const bool x_first = (kx > ky) || (kx == ky && ix < iy);
+            // segments with (x & k) == 0 end up in the output order
+            if (((x & k) == 0) != x_first) {
+              cand_key[x] = ky; cand_key[y] = kx;
+              cand_id[x] = iy; cand_id[y] = ix;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    for (int q = tid; q < k_sel; q += kThreads) {
+      const double kq = cand_key[q];
+      sort_id[q] = cand_id[q];
+      sort_s[q] = cov ? (invZ_ok != 0.0 ? __ddiv_rn(kq, Z) : 0.0) : kq;
+    }
   }
   __syncthreads();
 
@@ -359,6 +398,19 @@ size_t route_workspace_bytes(int H, int N, int M) {
   return ((size_t)H * N * M * sizeof(double) + 255) & ~(size_t)255;
 }
 
+// Candidate capacity: max(k_cov, k_unc), at least 1, rounded up to a power
+// of two when the bitonic sort is used.
+int route_kcap(int k_cov, int k_unc) {
+  int k = k_cov > k_unc ? k_cov : k_unc;
+  if (k < 1) k = 1;
+  if (k > kRankSortMax) {
+    int p = 1;
+    while (p < k) p <<= 1;
+    k = p;
+  }
+  return k;
+}
+
 size_t route_smem_bytes(int M, int kcap) {
   const int W = (M + 31) / 32;
   size_t b = (size_t)kcap * (8 + 8 + 4 + 4) + (size_t)W * 8;
@@ -385,8 +437,7 @@ cudaError_t launch_route(const float *p, const float *g, const uint8_t *covered,
   a.route_ids = route_ids; a.route_len = route_len; a.route_nbudget = route_nbudget;
   a.R_max = R_max;
   a.ws_keys = (M <= kSmemKeysMaxM) ? nullptr : static_cast<double *>(ws);
-  a.kcap = prm->k_cov > prm->k_unc ? prm->k_cov : prm->k_unc;
-  if (a.kcap < 1) a.kcap = 1;
+  a.kcap = route_kcap(prm->k_cov, prm->k_unc);
   a.dev_status = dev_status;
   const size_t smem = route_smem_bytes(M, a.kcap);
   cudaError_t e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
