@@ -341,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // score products without waiting for the PVs and the other way round.
     const int kk = nslot / 2;
     if (warp == 0 || warp == 2) {
-      // ================= TMA producers: warp 0 K (and Q), warp 2 V =================
+      // ================= TMA producers: warp 0 K, warp 2 V =================
       const bool is_k = warp == 0;
       if (lane == 0 && n > 0) {
         const CUtensorMap *hist_map = is_k ? &tmK : &tmV;
