@@ -265,8 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < kBufs; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], kChainThreads);
-      mbar_init(&p_full[b], kChainThreads);
+      mbar_init(&s_free[b], kChainThreads / 32);  // one arrival per warp
+      mbar_init(&p_full[b], kChainThreads / 32);
       mbar_init(&pv_done[b], 1);
     }
     mbar_init(x_fin, kSoftThreads);
@@ -462,7 +462,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int q = 0; q < 4; ++q) reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&sv[32 * q]));
       tc_fence_before();
-      mbar_arrive(&s_free[ch]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[ch]);
       float mx[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
@@ -539,7 +540,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       ref_own = ref;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[ch]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[ch]);
     }
     // epilogue: every MMA must be done before O is read and before the ring
     // (idle from then on) takes the row-sum exchange; mma_done completes once
