@@ -680,7 +680,8 @@ def _geometry_chain(layout: str = "gilbert", seed: int = 20261203):
            "cov": torch.empty(N, dtype=torch.uint8, device="cuda"),
            "st": torch.zeros(1, dtype=torch.int32, device="cuda"),
            "mw_ws": torch.empty(rbs.velox_multiwarp_workspace_size(len(src), T, H, W),
-                                dtype=torch.uint8, device="cuda")}
+                                dtype=torch.uint8, device="cuda"),
+           "cell": cell}
     B = buf
 
     def table():
@@ -731,6 +732,20 @@ def run_geometry(args):
     print(json.dumps(out), flush=True)
 
 
+def _route_union(route_ids: torch.Tensor, route_len: torch.Tensor) -> float:
+    """Mean over heads of the number of distinct tiles the head's routes
+    touch (the K/V tiles a launch must read at least once)."""
+    ids = route_ids.cpu().numpy()
+    lens = route_len.cpu().numpy()
+    total = 0
+    for h in range(ids.shape[0]):
+        seen = set()
+        for i in range(ids.shape[1]):
+            seen.update(ids[h, i, :lens[h, i]].tolist())
+        total += len(seen)
+    return total / max(1, ids.shape[0])
+
+
 def _route_runs(route_ids: torch.Tensor, route_len: torch.Tensor):
     """Mean route length and mean length of the runs of consecutive block
     ids in the routes (each route taken as a sorted set)."""
@@ -749,36 +764,59 @@ def run_layouts(args):
     """Gilbert against THW-linear token order through the whole routed path
     at the chunk-48 shape: the geometry chain of each order (slab tables from
     the same depth maps, multiwarp, g, coverage), then importance, route
-    build and attention on the same Q/K/V.  One JSON line per order: mean
-    route length, mean run of consecutive block ids in a route, attention
-    time.  `--layout` restricts it to one order (for an ncu capture)."""
+    build and attention.  Two input recipes: `random` (the N(0, 1) Q/K/V of
+    the bench, the same rows under both orders) and `positional` (Q/K from
+    synth.positional, whose q . k follows the distance between the tokens'
+    lattice positions, each token keeping its values under both orders; V
+    N(0, 1)).  One JSON line per order and recipe: mean route length, mean
+    run of consecutive block ids in a route, distinct tiles per head (the
+    K/V a launch must read), attention time.  `--layout` and `--qk` restrict
+    it (for an ncu capture)."""
     from routed_block_sparse_b200.pipeline import layer_for
     from synth import config, make_inputs
+    from synth.positional import positional_qk
 
     wl = config(3)
     if args.heads:
         from dataclasses import replace
         wl = replace(wl, heads=args.heads)
     inp = make_inputs(wl, "cuda")
+    T, Hl, Wl = wl.lattice
+    q0 = wl.q_chunk * T * Hl * Wl  # rank of the current chunk's first token
     for layout in (("gilbert", "thw") if args.layout == "both" else (args.layout,)):
         buf, calls, _ = _geometry_chain(layout)
         for _, fn in calls:
             fn()
-        layer = layer_for(wl, order=layout)
-        layer.importance(inp.Q, inp.K)
-        layer.route(buf["g"], buf["cov"])
-        torch.cuda.synchronize()
-        mean_len, mean_run = _route_runs(layer.route_ids, layer.route_len)
-        t_att = _time_us(lambda: layer.attend(inp.Q, inp.K, inp.V), reps=20)
-        tiles = float(layer.route_len.sum().item())
-        print(json.dumps({"layout": layout, "config": bench_config(wl),
-                          "g_nonzero_pairs": int((buf["g"] > 0).sum().item()),
-                          "covered_blocks": int(buf["cov"].sum().item()),
-                          "mean_route_len": mean_len, "mean_run_len": mean_run,
-                          "attn_us": t_att,
-                          "attn_tflops": 4.0 * 128 ** 3 * tiles / (t_att * 1e-6) / 1e12,
-                          "dev_status": layer.status() | int(buf["st"].item())}), flush=True)
-        del layer, buf
+        for qk in (("random", "positional") if args.qk == "both" else (args.qk,)):
+            if qk == "positional":
+                cell = buf["cell"]
+                Q, K = positional_qk(cell[q0:q0 + wl.n_q_blocks * wl.b],
+                                     cell[:wl.n_kv_blocks * wl.b], wl.heads, Hl, Wl,
+                                     cell.numel(), wl.d)
+            else:
+                Q, K = inp.Q, inp.K
+            layer = layer_for(wl, order=layout)
+            layer.importance(Q, K)
+            layer.route(buf["g"], buf["cov"])
+            torch.cuda.synchronize()
+            mean_len, mean_run = _route_runs(layer.route_ids, layer.route_len)
+            union = _route_union(layer.route_ids, layer.route_len)
+            t_att = _time_us(lambda: layer.attend(Q, K, inp.V), reps=20)
+            tiles = float(layer.route_len.sum().item())
+            print(json.dumps({"layout": layout, "qk": qk, "config": bench_config(wl),
+                              "g_nonzero_pairs": int((buf["g"] > 0).sum().item()),
+                              "covered_blocks": int(buf["cov"].sum().item()),
+                              "mean_route_len": mean_len, "mean_run_len": mean_run,
+                              "distinct_tiles_per_head": union,
+                              "attn_us": t_att,
+                              "attn_tflops": 4.0 * 128 ** 3 * tiles / (t_att * 1e-6) / 1e12,
+                              "dev_status": layer.status() | int(buf["st"].item())}),
+                  flush=True)
+            del layer
+            if qk == "positional":
+                del Q, K
+            torch.cuda.empty_cache()
+        del buf
         torch.cuda.empty_cache()
 
 
@@ -964,6 +1002,8 @@ def main():
     ap.add_argument("--layouts", action="store_true",
                     help="Gilbert vs THW-linear order through geometry, routes and attention")
     ap.add_argument("--layout", default="both", choices=["both", "gilbert", "thw"])
+    ap.add_argument("--qk", default="both", choices=["both", "random", "positional"],
+                    help="--layouts input recipe: random N(0,1) Q/K or positional Q/K")
     ap.add_argument("--heads", type=int, default=0,
                     help="run a reduced head count (profiler captures only)")
     args = ap.parse_args()
