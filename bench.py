@@ -541,14 +541,17 @@ def _graph_replay(step, steps, dev):
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize(dev)
-        a.record()
-        for _ in range(steps):
-            graph.replay()
-        b.record()
-        torch.cuda.synchronize(dev)
+        # timed after the eager loop, when the clock may have started to drop
+        # under the power cap: the median SM clock of this loop is reported
+        with ClockSampler(dev) as clocks:
+            a.record()
+            for _ in range(steps):
+                graph.replay()
+            b.record()
+            torch.cuda.synchronize(dev)
         ms = a.elapsed_time(b) / steps
         del graph
-        return {"ms_per_step": ms, "steps": steps}
+        return {"ms_per_step": ms, "steps": steps, "sm_mhz": clocks.summary()["sm_mhz"]}
     except Exception as e:  # reported, not fatal: the eager numbers stand alone
         return {"error": str(e)[:200]}
 
