@@ -141,3 +141,31 @@ def test_token_on_a_rectangle_edge_is_marginal():
     # units at depth 4; (1.5, 3) and (1.99, 3): outside by 0.5 and 0.01
     # tokens (1 and 0.02 world units): both clear of the margin
     assert (n[0], lo[0], hi[0]) == (2, 1, 2)
+
+
+def test_coverage_count_faces_half_open_rectangle_closed_depth():
+    # The coverage count of a token on each face of SLAB, with exactly
+    # representable coordinates (fx = 2, cx = 4, R = I: token (u, v, z)
+    # projects back to (u, v) at depth z with no rounding): the rectangle is
+    # [u0, u1) x [v0, v1), the depth interval [z-, z+].
+    c = cam()
+    faces = [((2.0, 3.0, 4.0), True),    # u = u0
+             ((6.0, 3.0, 4.0), False),   # u = u1
+             ((3.0, 2.0, 4.0), True),    # v = v0
+             ((3.0, 6.0, 4.0), False),   # v = v1
+             ((3.0, 3.0, 3.0), True),    # z = z-
+             ((3.0, 3.0, 5.0), True)]    # z = z+
+    uvz = np.array([[t for t, _ in faces]], dtype=np.float32).reshape(len(faces), 1, 3)
+    n, _, _ = geo.coverage_bounds([c], [0] * len(faces), uvz, [0], [SLAB], [1])
+    assert n.tolist() == [int(want) for _, want in faces]
+    for (u, v, z), want in faces:
+        assert geo.token_inside(c, u, v, z, c, SLAB) == want
+
+
+def test_covered_when_rho_equals_eta():
+    # rho = 2 / 4 = eta = 0.5 exactly: covered (rho >= eta)
+    uvz = np.zeros((1, 4, 3), dtype=np.float32)
+    uvz[0, :, :2] = 3.0
+    uvz[0, :, 2] = [4.0, 4.0, 9.0, 9.0]
+    rho, cov = geo.coverage([cam()], [0], uvz, [0], [SLAB], [1], eta=0.5)
+    assert rho.tolist() == [0.5] and cov.tolist() == [1]

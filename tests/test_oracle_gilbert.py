@@ -238,3 +238,16 @@ def test_gilbert_keeps_adjacent_tokens_in_one_block_more_often_than_thw():
     fg = _same_block_fraction(bg.reshape(H, W))
     ft = _same_block_fraction(bt.reshape(H, W))
     assert fg > ft + 0.1
+
+
+@pytest.mark.parametrize("T,H,W", [(3, 3, 4), (4, 4, 8), (2, 32, 48)])
+def test_first_frame_is_the_plain_curve_and_odd_frames_its_mirror(T, H, W):
+    # mirror *alternate* frames starting from the plain map: frame 0 is the
+    # frame curve itself (from cell (0, 0) to (W-1, 0)), frame 1 its mirror
+    rank, cell, _ = gilbert.global_order(T, H, W, 2, 1)
+    r = rank.reshape(2 * T, H, W)
+    r2 = gilbert.frame_rank_map(W, H)
+    assert np.array_equal(r[0], r2)
+    assert np.array_equal(r[1] - H * W, r2[:, ::-1])
+    assert int(cell[0]) == 0 and r[0][0, W - 1] == H * W - 1
+    assert r[1][0, W - 1] == H * W and r[1][0, 0] == 2 * H * W - 1

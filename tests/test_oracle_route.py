@@ -204,3 +204,15 @@ def test_ties_at_the_cut_go_to_lower_ids():
     g[[30, 12, 20]] = [0.2, 1.0, 0.5]
     budget, _, _ = rt.route_row(p, g, True, rt.Params(k_cov=7, theta_cov=2.0), 35, 5)
     assert budget == [12, 20, 35, 36, 37, 38, 39]
+
+
+def test_cut_when_mass_reaches_theta_exactly():
+    # dyadic masses and theta, all exact in fp32 and fp64: the prefix stops at
+    # the first block whose cumulative mass reaches theta (>=), not after it
+    p = np.array([0.0625, 0.5, 0.125, 0.25, 0.0625], dtype=np.float32)
+    g = np.zeros(5, dtype=np.float32)
+    prm = rt.Params(theta_unc=0.75, k_unc=5)
+    budget, extras, info = rt.route_row(p, g, False, prm, 0, 0)
+    assert budget == [1, 3] and extras == [] and info["mass_at_cut"] == 0.75
+    prm = rt.Params(theta_unc=0.875, k_unc=5)
+    assert rt.route_row(p, g, False, prm, 0, 0)[0] == [1, 2, 3]

@@ -166,3 +166,16 @@ def test_warp_sample_closed_form():
     # behind the target camera: no landing
     cell, depth, _, _ = osl.warp_sample(cam(), cam(C=(0.0, 0.0, 5.0)), 4.5, 2.5, 4.0, 4, 8)
     assert cell is None and depth < 0
+
+
+def test_slab_needs_exactly_n_min_reliable_samples():
+    # block 0 has exactly n_min reliable samples (valid), block 1 one fewer
+    T, H, W, b, nc = 1, 2, 4, 4, 1
+    _, cell, _ = gilbert.thw_linear_order(T, H, W, nc, b)
+    depth = np.full((1, H, W), 2.0, dtype=np.float32)
+    mask = np.ones(depth.shape, dtype=np.uint8)
+    mask[0, 1, 0] = 0                     # row 1 (block 1): 3 reliable samples
+    slab, _, valid = osl.slab_table(depth, None, mask, cell, H, W, b, 0, 0, 2,
+                                    osl.SlabParams(s=1, n_min=4))
+    assert valid.tolist() == [1, 0]
+    assert slab[0].tolist() == [0.0, 4.0, 0.0, 1.0, 2.0, 2.0]
