@@ -182,3 +182,23 @@ def check_multiwarp(zq_gpu, zq_ref, unsure):
     n_uns = int(unsure.sum())
     assert n_uns <= max(2, UNSURE_FRAC * unsure.size), f"{n_uns} unsure tokens"
     return n_uns
+
+
+def routes_from_gpu_p(layer, wl, g, covered, nbr):
+    """Oracle routes of every (head, query block) row from the GPU's own p
+    (the route step's input), compared with the GPU routes: bit-exact except
+    at a mass cut within MASS_EPS of theta.  Returns ({(h, i): tile list},
+    number of rows that differ at the cut)."""
+    prm = oracle_params(wl.params)
+    p = layer.p.cpu().numpy()
+    g, cov = g.cpu().numpy(), covered.cpu().numpy()
+    rid, rlen, rnb = layer.route_ids.cpu(), layer.route_len.cpu(), layer.route_nbudget.cpu()
+    out, n_cut = {}, 0
+    for h in range(wl.heads):
+        for i in range(wl.n_q_blocks):
+            ref = ort.route_row(p[h, i], g[i], bool(cov[i]), prm, wl.prev_begin,
+                                wl.prev_count, list(nbr[i]))
+            gpu = gpu_row(rid, rlen, rnb, h, i)
+            n_cut += check_route_row(gpu, ref, f"head {h} row {i}") == "cut"
+            out[(h, i)] = gpu[0] + gpu[1]
+    return out, n_cut

@@ -14,7 +14,7 @@ from oracle import gilbert
 from routed_block_sparse_b200.pipeline import layer_for
 from synth import config, make_inputs, sweep_workload
 from parity import (assert_attention_close, attention_rows, f64, gpu_row, oracle_importance,
-                    oracle_params, oracle_routes)
+                    oracle_params, oracle_routes, routes_from_gpu_p)
 
 pytestmark = pytest.mark.gpu
 
@@ -91,28 +91,6 @@ def test_pipeline_sweep_and_dense(lib):
         torch.cuda.empty_cache()
 
 
-def _routes_from_gpu_p(layer, inp, nbr):
-    """Oracle routes of every (head, query block) row from the GPU's own p
-    (the route step's input), compared with the GPU routes: bit-exact except
-    at a mass cut within MASS_EPS of theta.  Returns {(h, i): tile list}."""
-    from oracle import route as ort
-    from parity import check_route_row
-    wl = inp.wl
-    prm = oracle_params(wl.params)
-    p = layer.p.cpu().numpy()
-    g, cov = inp.g.cpu().numpy(), inp.covered.cpu().numpy()
-    rid, rlen, rnb = layer.route_ids.cpu(), layer.route_len.cpu(), layer.route_nbudget.cpu()
-    out, n_cut = {}, 0
-    for h in range(wl.heads):
-        for i in range(wl.n_q_blocks):
-            ref = ort.route_row(p[h, i], g[i], bool(cov[i]), prm, wl.prev_begin,
-                                wl.prev_count, list(nbr[i]))
-            gpu = gpu_row(rid, rlen, rnb, h, i)
-            n_cut += check_route_row(gpu, ref, f"head {h} row {i}") == "cut"
-            out[(h, i)] = gpu[0] + gpu[1]
-    return out, n_cut
-
-
 @pytest.mark.slow
 def test_pipeline_forty_layers(lib):
     """The 40-layer workload (per-layer seeds, regenerated into reused
@@ -132,7 +110,7 @@ def test_pipeline_forty_layers(lib):
         layer.forward(inp.Q, inp.K, inp.V, inp.g, inp.covered)
         torch.cuda.synchronize()
         assert layer.status() == 0, f"layer {li}"
-        routes, n_cut = _routes_from_gpu_p(layer, inp, nbr)
+        routes, n_cut = routes_from_gpu_p(layer, wl, inp.g, inp.covered, nbr)
         assert n_cut <= 2, f"layer {li}: {n_cut} rows differ at the cut"
         heads = [(li + 10 * k) % 40 for k in range(4)]
         for h, ph in oracle_importance(inp.Q, inp.K, heads).items():
