@@ -196,3 +196,27 @@ def test_longest_route_the_abi_allows(lib):
     assert st == 0
     ref = attention_rows(inp.Q, inp.K, inp.V, sorted(routes), lambda h, i: routes[(h, i)])
     assert_attention_close(O, lse, ref)
+
+
+@pytest.mark.slow
+def test_routes_at_the_largest_cache_the_abi_allows(lib):
+    # M = VELOX_MAX_BLOCKS = 65536 history blocks (2 GB each of K and V for one
+    # head): the compaction bitmap is full, tile coordinates reach
+    # 65535 * 128.  The oracle sees only the tiles a row lists (attention over
+    # the listed tiles is the whole computation), gathered on the device.
+    H, N, M = 1, 3, 65536
+    inp = make_inputs(small(H, N, M, 0), "cuda")
+    routes = {(0, 0): [0, 1, 32768, 65534, 65535],
+              (0, 1): [65535],
+              (0, 2): list(range(65536 - 300, 65536, 3))}
+    R_max = 128
+    rid, rlen = _routes_tensor(routes, H, N, R_max)
+    O, lse, st = _attend(inp, rid, rlen, R_max)
+    assert st == 0
+    for (h, i), tiles in routes.items():
+        idx = torch.cat([torch.arange(t * 128, (t + 1) * 128) for t in tiles]).cuda()
+        Ks, Vs = inp.K[h:h + 1, idx], inp.V[h:h + 1, idx]
+        Qs = inp.Q[h:h + 1, i * 128:(i + 1) * 128]
+        ref = attention_rows(Qs, Ks, Vs, [(0, 0)], lambda _h, _i: range(len(tiles)))
+        assert_attention_close(O[h:h + 1, i * 128:(i + 1) * 128], lse[h:h + 1, i * 128:(i + 1) * 128],
+                               ref)
