@@ -236,3 +236,15 @@ def test_route_bad_safeguard_ids_are_flagged(lib):
     for i in range(N):
         ids = rid[0, i, :int(rl[0, i])].tolist()
         assert all(0 <= x < M for x in ids) and len(set(ids)) == len(ids)
+
+
+def test_route_at_the_largest_history_and_cap(lib):
+    # M = VELOX_MAX_BLOCKS = 65536 (keys in the workspace), caps at
+    # VELOX_MAX_ROUTE = 4096 (the bitonic sort over 4096 survivors); covered
+    # rows take the threshold above 1 (the cap binds), uncovered rows 0.9 on
+    # peaked importance
+    H, N, M = 1, 3, 65536
+    p32 = _synthetic_p(H, N, M, 9, peaked=4.0)
+    g, cov = _geom(N, M, 9)
+    prm = rbs.route_params(theta_cov=2.0, theta_unc=0.9, k_cov=4096, k_unc=4096)
+    _run_case(p32, g, cov, prm, M - 48, 48)
