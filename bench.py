@@ -518,6 +518,16 @@ def run_velox(args, world, rank, local):
     # the same step captured once as a CUDA graph and replayed (the seven
     # launches go out as one graph launch); reported beside the eager timing
     line["graph"] = _graph_replay(step, args.steps, dev)
+    # the SM clock inside the attention kernel, measured from the GPU (after
+    # the timed region): NVML's sampled clock does not show the power limiter
+    eff = _attn_effective_clock(layer, inp, dev, stream)
+    if eff is not None:
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        line["roofline"]["effective_sm_mhz"] = eff
+        line["roofline"]["attn_cycles_per_tile_per_sm"] = attn_ms * 1e3 * eff * sms / tiles
+        line["roofline"]["effective_clock_source"] = (
+            "velox_clock_probe (one CTA, clock64 against %globaltimer every 2 us) on a side "
+            "stream beside 5 attention calls after the timed region; middle half of their span")
 
     # end to end through the public API with host buffers
     if args.e2e_steps > 0:
@@ -529,6 +539,34 @@ def run_velox(args, world, rank, local):
                                 "sample_seconds": r["sample_s"]}
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def _attn_effective_clock(layer, inp, dev, stream, calls=5, n=6000, pause_ns=2000):
+    """Median SM clock (MHz) while `calls` attention calls run back to back,
+    from the clock probe on a side stream; None if it cannot be read."""
+    import routed_block_sparse_b200 as rbs
+    try:
+        samples = torch.zeros(n, 2, dtype=torch.int64, device=dev)
+        side = torch.cuda.Stream(dev)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        rbs.velox_clock_probe(samples, n, pause_ns, stream=side)
+        a.record(stream)
+        for _ in range(calls):
+            layer.attend(inp.Q, inp.K, inp.V, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        span_ns = a.elapsed_time(b) * 1e6
+        x = samples.cpu().numpy().astype(np.float64)
+        c, t = x[:, 0], x[:, 1]
+        rate = np.diff(c) / np.maximum(np.diff(t), 1.0)
+        mid = (t[1:] >= t[0] + 0.25 * span_ns) & (t[1:] <= t[0] + 0.75 * span_ns)
+        if not mid.any():
+            return None
+        return float(np.median(rate[mid]) * 1e3)
+    except Exception:
+        return None
 
 
 def _graph_replay(step, steps, dev):

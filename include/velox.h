@@ -24,8 +24,9 @@
  * velox_multiwarp (the history-side geometry: frustum slabs from depth maps,
  * the recency-priority multiwarp depth of the current frames),
  * velox_route_schedule (longest-route-first row order),
- * velox_block_importance_noalloc and velox_wait_selftest (the bounded waits
- * driven to their limit).
+ * velox_block_importance_noalloc, velox_wait_selftest (the bounded waits
+ * driven to their limit) and velox_clock_probe (the SM clock seen from
+ * inside the GPU, for measurement).
  *
  * Conventions shared by every call
  * --------------------------------
@@ -114,7 +115,7 @@ typedef struct {
 /* Human-readable text of a status; never NULL. */
 VELOX_API const char *velox_status_string(velox_status s);
 
-/* ABI version of this header (major * 100 + minor): 103. */
+/* ABI version of this header (major * 100 + minor): 104. */
 VELOX_API int velox_abi_version(void);
 
 /*
@@ -527,6 +528,20 @@ VELOX_API velox_status velox_multiwarp_workspace_size(int S, int n_tgt, int H, i
  */
 VELOX_API velox_status velox_wait_selftest(int limit_us, int32_t *dev_status,
                                            int64_t *elapsed_ns, velox_stream_t stream);
+
+/*
+ * velox_clock_probe -- sample the SM clock against the global timer.
+ *
+ * The pages have no counterpart: this is a measurement aid.  One CTA of one
+ * warp; its thread 0 writes n pairs {clock64(), %globaltimer ns} to samples
+ * (device, [n][2] int64), pausing about pause_ns nanoseconds between pairs.
+ * Launched on its own stream beside another kernel, the ratio of successive
+ * differences (cycles per ns) is the SM clock in GHz while that kernel runs
+ * (the power limiter can hold it far below the clock the driver reports).
+ * 1 <= n <= 1,000,000 and pause_ns <= 1,000,000, else VELOX_ERR_INVALID_ARG.
+ */
+VELOX_API velox_status velox_clock_probe(int64_t *samples, int n, int pause_ns,
+                                         velox_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -47,7 +47,7 @@ EXPORTS = ("velox_status_string", "velox_abi_version", "velox_gilbert_order",
            "velox_route_schedule", "velox_two_phase_attn", "velox_slab_overlap",
            "velox_coverage", "velox_route_audit", "velox_thw_linear_order",
            "velox_slab_table", "velox_multiwarp", "velox_multiwarp_workspace_size",
-           "velox_wait_selftest")
+           "velox_wait_selftest", "velox_clock_probe")
 
 
 class VeloxError(RuntimeError):
@@ -110,6 +110,8 @@ def _load() -> ctypes.CDLL:
                                          P]
     lib.velox_wait_selftest.restype = I
     lib.velox_wait_selftest.argtypes = [I, P, P, P]
+    lib.velox_clock_probe.restype = I
+    lib.velox_clock_probe.argtypes = [P, I, I, P]
     return lib
 
 
@@ -367,6 +369,12 @@ def velox_multiwarp(cams, n_cams, src_depth, src_cam, S, tgt_cam, n_tgt, H, W, s
                               _arg(zq, "zq", F32, _n(n_tgt, H, W)), _ptr(ws), _nbytes(ws),
                               _arg(dev_status, "dev_status", I32, 1), _stream(stream))
     _check("velox_multiwarp", st)
+
+
+def velox_clock_probe(samples, n, pause_ns=2000, stream=None):
+    st = _lib.velox_clock_probe(_arg(samples, "samples", (torch.int64,), _n(n, 2)), int(n),
+                                int(pause_ns), _stream(stream))
+    _check("velox_clock_probe", st)
 
 
 def velox_wait_selftest(limit_us, dev_status, elapsed_ns=None, stream=None):

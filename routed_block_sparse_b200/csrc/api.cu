@@ -56,6 +56,7 @@ cudaError_t launch_multiwarp(const velox_camera *cams, int n_cams, const float *
 cudaError_t launch_audit(const float *p, const float *g, int H, int N, int M, double lam,
                          double tau, double g_ref, int k_geo, int k_fuse, int32_t *counts,
                          cudaStream_t stream);
+cudaError_t launch_clock_probe(int64_t *samples, int n, uint32_t pause_ns, cudaStream_t stream);
 cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t *dev_status, int64_t *elapsed_ns,
                                  cudaStream_t stream);
 }  // namespace velox
@@ -116,7 +117,7 @@ const char *velox_status_string(velox_status s) {
   return "unknown status";
 }
 
-int velox_abi_version(void) { return 103; }
+int velox_abi_version(void) { return 104; }
 
 }  // extern "C"
 
@@ -411,6 +412,15 @@ velox_status velox_multiwarp(const velox_camera *cams, int n_cams, const float *
   return from_cuda(velox::launch_multiwarp(cams, n_cams, src_depth, src_cam, S, tgt_cam, n_tgt, H,
                                            W, s, k_warp, zq, ws, dev_status,
                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+velox_status velox_clock_probe(int64_t *samples, int n, int pause_ns, velox_stream_t stream) {
+  if (!samples || n < 1 || n > 1000000 || pause_ns < 0 || pause_ns > 1000000)
+    return VELOX_ERR_INVALID_ARG;
+  velox_status st = check_device();
+  if (st != VELOX_OK) return st;
+  return from_cuda(velox::launch_clock_probe(samples, n, static_cast<uint32_t>(pause_ns),
+                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
 velox_status velox_wait_selftest(int limit_us, int32_t *dev_status, int64_t *elapsed_ns,

@@ -60,7 +60,7 @@ def test_binding_names_match_header(built):
 
 def test_status_strings_and_version(built):
     import routed_block_sparse_b200 as rbs
-    assert rbs.velox_abi_version() == 103
+    assert rbs.velox_abi_version() == 104
     for s in range(8):
         assert isinstance(rbs.velox_status_string(s), str) and rbs.velox_status_string(s)
     assert rbs.velox_status_string(99) == "unknown status"
@@ -154,3 +154,14 @@ def test_wait_selftest_arguments_checked_on_the_host(built):
     assert lib.velox_wait_selftest(1000, None, None, None) == 1
     for bad in (0, -1, 2_000_001):
         assert lib.velox_wait_selftest(bad, fake, None, None) == 1
+
+
+def test_clock_probe_arguments_checked_on_the_host(built):
+    lib = ctypes.CDLL(built)
+    lib.velox_clock_probe.restype = ctypes.c_int
+    fake = ctypes.c_void_p(0x10000)
+    assert lib.velox_clock_probe(None, 10, 100, None) == 1
+    for n, pause in ((0, 100), (-1, 100), (1_000_001, 100), (10, -1), (10, 1_000_001)):
+        assert lib.velox_clock_probe(fake, n, pause, None) == 1
+    # valid arguments, no sm_100 device: refused, nothing runs
+    assert lib.velox_clock_probe(fake, 10, 100, None) == 5

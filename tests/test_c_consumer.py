@@ -20,7 +20,7 @@ C_SOURCE = r"""
 
 int main(void) {
   size_t ws = 0, mw = 0;
-  if (velox_abi_version() != 103) return 1;
+  if (velox_abi_version() != 104) return 1;
   if (velox_workspace_size(40, 48, 2256, 128, &ws) != VELOX_OK || ws == 0) return 2;
   if (velox_multiwarp_workspace_size(60, 4, 32, 48, &mw) != VELOX_OK) return 3;
   if (mw != (size_t)4 * 60 * 4 * 32 * 48) return 4;
@@ -53,4 +53,4 @@ def test_c99_program_links_and_calls_the_library(tmp_path):
     assert cc.returncode == 0, cc.stderr
     run = subprocess.run([str(exe)], capture_output=True, text=True)
     assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
-    assert run.stdout.split()[0] == "103"
+    assert run.stdout.split()[0] == "104"
