@@ -140,11 +140,12 @@ __global__ void __launch_bounds__(256) logits_kernel(const float *__restrict__ q
   }
 }
 
-// Fused K pooling + logits.  Grid-stride over chunks of kFusedBlocks key
-// blocks of one head (chunk c: head c / cpr, blocks (c % cpr) * kFusedBlocks ..),
-// 256 threads, grid sized to the resident capacity.
-// Warp w of a CTA streams the 8 consecutive key blocks r0 + 8w .. r0 + 8w + 7
-// with no block-level barrier after the qbar load.  After the half-warp
+// Fused K pooling + logits.  Grid-stride over chunks of 8 * per_warp key
+// blocks of one head (chunk c: head c / cpr, blocks (c % cpr) * 8 * per_warp
+// ..), 256 threads, grid sized to the resident capacity; per_warp is 8 unless
+// H * M is too small to give every CTA slot a chunk.
+// Warp w of a CTA streams the per_warp consecutive key blocks r0 + w per_warp
+// .. with no block-level barrier after the qbar load.  After the half-warp
 // exchange both halves hold the 8 channel sums of lane (l & 15); half-warp 0
 // computes the logits of query rows 0, 2, 4, ... and half-warp 1 of rows
 // 1, 3, 5, ..., each as 8 products plus a 16-lane shuffle reduction, staged
@@ -152,13 +153,12 @@ __global__ void __launch_bounds__(256) logits_kernel(const float *__restrict__ q
 // (8 consecutive logits = 32 bytes per row) once the warp's blocks are done.
 constexpr int kFusedMaxN = 96;
 constexpr int kFusedWarps = 8;
-constexpr int kFusedPerWarp = 8;
-constexpr int kFusedBlocks = kFusedWarps * kFusedPerWarp;  // key blocks per CTA
+constexpr int kFusedPerWarp = 8;  // most key blocks per warp (the staging width)
 
 __global__ void __launch_bounds__(256) pool_logits_kernel(const uint16_t *__restrict__ K,
                                                           const float *__restrict__ qbar, int H,
                                                           int N, int M, float scale,
-                                                          float *__restrict__ p) {
+                                                          int per_warp, float *__restrict__ p) {
   extern __shared__ float4 fsm[];
   float *qs = reinterpret_cast<float *>(fsm);  // [N][D] means of the chunk's head
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -166,15 +166,16 @@ __global__ void __launch_bounds__(256) pool_logits_kernel(const uint16_t *__rest
   const int col = (lane & 15) * 8;
   const int row0 = lane >> 4;
   const float cs = scale * (1.0f / BT);  // logit = scale * qbar . (sum / b)
-  const int cpr = (M + kFusedBlocks - 1) / kFusedBlocks;
+  const int per_cta = kFusedWarps * per_warp;  // key blocks per chunk (per_warp <= 8)
+  const int cpr = (M + per_cta - 1) / per_cta;
   for (int c = blockIdx.x; c < H * cpr; c += gridDim.x) {
   const int h = c / cpr;
   __syncthreads();  // every warp is done with the previous chunk's qbar
   for (int e = threadIdx.x; e < N * D / 4; e += blockDim.x)
     fsm[e] = reinterpret_cast<const float4 *>(qbar + (size_t)h * N * D)[e];
   __syncthreads();
-  const int rw = (c - h * cpr) * kFusedBlocks + warp * kFusedPerWarp;  // first block of the warp
-  for (int k = 0; k < kFusedPerWarp; ++k) {
+  const int rw = (c - h * cpr) * per_cta + warp * per_warp;  // first block of the warp
+  for (int k = 0; k < per_warp; ++k) {
     const int rb = rw + k;
     if (rb >= M) break;  // uniform across the warp
     float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -205,7 +206,7 @@ __global__ void __launch_bounds__(256) pool_logits_kernel(const uint16_t *__rest
     }
   }
   __syncwarp();
-  const int nb = min(kFusedPerWarp, M - rw);
+  const int nb = min(per_warp, M - rw);
   for (int e = lane; e < N * kFusedPerWarp; e += 32) {
     const int i = e / kFusedPerWarp, k = e - i * kFusedPerWarp;
     if (k < nb) p[((size_t)h * N + i) * M + rw + k] = lg[e];
@@ -285,11 +286,26 @@ cudaError_t launch_importance(const uint16_t *Q, const uint16_t *K, int H, int N
                                (int)smem);
       if (e != cudaSuccess) return e;
     }
-    const int chunks = H * ((M + kFusedBlocks - 1) / kFusedBlocks);
     int per_sm = (int)((220 * 1024) / (smem + 1024));
     per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
-    const int grid_f = chunks < 148 * per_sm ? chunks : 148 * per_sm;
-    pool_logits_kernel<<<grid_f, 256, smem, stream>>>(K, qbar, H, N, M, scale, p);
+    // key blocks per warp: the count (1..8) whose busiest CTA streams the
+    // fewest blocks, i.e. ceil(chunks / slots) * per_warp smallest, the larger
+    // count on ties -- 8 at the chunk-48 shape, fewer when a few heads would
+    // leave CTA slots empty
+    const long long slots = 148LL * per_sm;
+    int per_warp = kFusedPerWarp;
+    long long best = -1;
+    for (int pw = kFusedPerWarp; pw >= 1; --pw) {
+      const long long ch = (long long)H * ((M + kFusedWarps * pw - 1) / (kFusedWarps * pw));
+      const long long cost = (ch + slots - 1) / slots * pw;
+      if (best < 0 || cost < best) {
+        best = cost;
+        per_warp = pw;
+      }
+    }
+    const int chunks = H * ((M + kFusedWarps * per_warp - 1) / (kFusedWarps * per_warp));
+    const int grid_f = chunks < slots ? chunks : (int)slots;
+    pool_logits_kernel<<<grid_f, 256, smem, stream>>>(K, qbar, H, N, M, scale, per_warp, p);
   } else {
     dim3 lg((M + LG_R - 1) / LG_R, H);
     logits_kernel<<<lg, 256, 0, stream>>>(qbar, kbar, N, M, scale, p);

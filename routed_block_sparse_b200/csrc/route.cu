@@ -11,8 +11,9 @@
 // One CTA per (head, query block) row:
 //   1. fused weights w_r in fp64 (explicit round-to-nearest operations, so
 //      no contraction changes the value), row sum Z;
-//   2. radix select (8 passes of 8 bits over an order-preserving 64-bit key)
-//      of the k largest non-reserved weights, ties to the lower id;
+//   2. radix select (passes of 8 bits over an order-preserving 64-bit key,
+//      from the highest byte in which the eligible keys differ) of the k
+//      largest non-reserved weights, ties to the lower id;
 //   3. rank sort of the <= k survivors (weight desc, id asc);
 //   4. warp scan of the normalised mass from the reserved mass on: the cut is
 //      the first position at which the mass before it reaches theta;
@@ -94,12 +95,15 @@ __device__ int block_excl_scan(int v, int *scratch, int *total) {
   return before + incl - v;
 }
 
-__global__ void __launch_bounds__(kThreads) route_kernel(RouteArgs a) {
+// six rows per SM: the register cap (40) costs a few bytes of spills and
+// keeps 2.2 waves at the chunk-48 shape instead of 3.2
+__global__ void __launch_bounds__(kThreads, 6) route_kernel(RouteArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ double s_dred[kWarps];
   __shared__ int s_ired[kWarps];
   __shared__ int s_hist[256];
   __shared__ int s_digit, s_greater, s_equal, s_ntake;
+  __shared__ uint64_t s_kand[kWarps], s_kor[kWarps];
 
   const int row = blockIdx.x;
   const int i = row % a.N;
@@ -128,22 +132,37 @@ __global__ void __launch_bounds__(kThreads) route_kernel(RouteArgs a) {
   for (int k = tid; k < W; k += kThreads) { bud_bits[k] = 0u; ext_bits[k] = 0u; }
 
   // ---- 1. fused weights and their sum
+  // loads four deep per thread (the same ids and summation order as a plain
+  // strided loop): one memory round trip per four keys
   double zpart = 0.0;
-  for (int r = tid; r < M; r += kThreads) {
-    const double pv = static_cast<double>(prow[r]);
-    double w = pv;
-    if (cov) {
-      const double gv = static_cast<double>(grow[r]);
-      double gh = 0.0;
-      if (gv > a.tau) {
-        gh = __ddiv_rn(gv, a.g_ref);
-        if (gh > 1.0) gh = 1.0;
-      }
-      w = __dmul_rn(pv, __dadd_rn(1.0, __dmul_rn(a.lam, gh)));
+  constexpr int kBatch = 4;
+  for (int base = tid; base < M; base += kThreads * kBatch) {
+    float pf[kBatch], gf[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int r = base + u * kThreads;
+      pf[u] = r < M ? __ldg(prow + r) : 0.f;
+      gf[u] = (cov && r < M) ? __ldg(grow + r) : 0.f;
     }
-    w = __dadd_rn(w, 0.0);  // -0 -> +0, so that zeros tie exactly
-    keys[r] = w;
-    zpart += w;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int r = base + u * kThreads;
+      if (r >= M) break;
+      const double pv = static_cast<double>(pf[u]);
+      double w = pv;
+      if (cov) {
+        const double gv = static_cast<double>(gf[u]);
+        double gh = 0.0;
+        if (gv > a.tau) {
+          gh = __ddiv_rn(gv, a.g_ref);
+          if (gh > 1.0) gh = 1.0;
+        }
+        w = __dmul_rn(pv, __dadd_rn(1.0, __dmul_rn(a.lam, gh)));
+      }
+      w = __dadd_rn(w, 0.0);  // -0 -> +0, so that zeros tie exactly
+      keys[r] = w;
+      zpart += w;
+    }
   }
   const double Z = cov ? block_sum(zpart, s_dred) : 1.0;
   const double invZ_ok = (Z > 0.0) ? 1.0 : 0.0;  // Z == 0: no mass ever counts
@@ -166,7 +185,41 @@ __global__ void __launch_bounds__(kThreads) route_kernel(RouteArgs a) {
   int need = k_sel;
   const bool select_all = (k_sel == n_elig);
   if (k_sel > 0 && !select_all) {
-    for (int shift = 56; shift >= 0; shift -= 8) {
+    // bytes that every eligible key shares decide nothing: start below them
+    uint64_t kand = ~0ull, kor = 0ull;
+    for (int r = tid; r < M; r += kThreads) {
+      if (r >= pb && r < pe) continue;
+      const uint64_t u = order_key(keys[r]);
+      kand &= u;
+      kor |= u;
+    }
+    const uint32_t a_hi = __reduce_and_sync(0xffffffffu, (uint32_t)(kand >> 32));
+    const uint32_t a_lo = __reduce_and_sync(0xffffffffu, (uint32_t)kand);
+    const uint32_t o_hi = __reduce_or_sync(0xffffffffu, (uint32_t)(kor >> 32));
+    const uint32_t o_lo = __reduce_or_sync(0xffffffffu, (uint32_t)kor);
+    if ((tid & 31) == 0) {
+      s_kand[tid >> 5] = ((uint64_t)a_hi << 32) | a_lo;
+      s_kor[tid >> 5] = ((uint64_t)o_hi << 32) | o_lo;
+    }
+    __syncthreads();
+    uint64_t all_and = ~0ull, all_or = 0ull;
+    for (int w = 0; w < kWarps; ++w) {
+      all_and &= s_kand[w];
+      all_or |= s_kor[w];
+    }
+    const uint64_t diff = all_and ^ all_or;
+    int shift0;
+    if (diff == 0ull) {
+      shift0 = -8;  // every eligible key is equal: all of them tie
+      mask = ~0ull;
+      prefix = all_and;
+    } else {
+      const int hb = 63 - __clzll(static_cast<long long>(diff));
+      shift0 = (hb >> 3) << 3;
+      mask = (shift0 >= 56) ? 0ull : ~((1ull << (shift0 + 8)) - 1ull);
+      prefix = all_and & mask;
+    }
+    for (int shift = shift0; shift >= 0; shift -= 8) {
       for (int k = tid; k < 256; k += kThreads) s_hist[k] = 0;
       __syncthreads();
       // warp-aggregated: keys mostly share their leading digits, so one
