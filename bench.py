@@ -9,10 +9,14 @@ larger than L2 (K + V = 5.9 GB), so no L2 flush is needed between steps.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl velox|reference]
 
 Prints one JSON line.  value = routed-attention FLOPs of the step (4 b^2 d per
-routed tile, from the actual route lengths) over the step time, summed over
-ranks (weak scaling: every rank runs its own layer; there is no data-path
-collective).  Per-call times, the roofline of the attention kernel, an
-end-to-end number through host buffers and the CPU oracle baseline are added.
+routed tile, from the actual route lengths), summed over ranks, over the
+slowest rank's step time.  With N ranks the heads of the one layer are split
+across them (strong scaling; `--shard layers` gives every rank its own layer
+instead); there is no data-path collective.  Per-call times, the roofline of
+the attention kernel (with the SM clock measured from the GPU beside the
+attention calls: the driver's sampled clock does not show the power
+limiter), an end-to-end number through host buffers and the CPU oracle
+baseline are added.
 """
 
 from __future__ import annotations
