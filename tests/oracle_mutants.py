@@ -10,6 +10,12 @@ fails.  The mistakes are planted on the CPU, in the oracle, never in the CUDA
 path.
 
 Entry: (name, oracle module, exact text, replacement, pin test file).
+
+Not listed because no pin can tell them apart from the oracle: changes of the
+Gilbert construction's split rule (for example a two-way split whenever the
+major edge is longer) that still give a unit-step curve from (0, 0) to
+(W-1, 0); the exact curve beyond its invariants is unpinned against the
+authors' figures, whose ranks are not in the text.
 """
 
 from __future__ import annotations
@@ -214,6 +220,61 @@ def thw_linear_order""", "test_oracle_gilbert.py"),
     ("audit: recall against the geometry's own top-K", "oracle.audit",
      "len(pos & a_geo), len(g_geo & a_geo)", "len(pos & g_geo), len(g_geo & a_geo)",
      "test_oracle_audit.py"),
+    # ---- marginal-decision bounds (the GPU parity rule's ranges)
+    ("geometry: marginal lower count includes the face band", "oracle.geometry",
+     "n_lo = int(np.count_nonzero(margin > eps))", "n_lo = int(np.count_nonzero(margin >= -eps))",
+     "test_oracle_geometry.py"),
+    ("geometry: marginal upper count drops the face band", "oracle.geometry",
+     "n_hi = int(np.count_nonzero(margin >= -eps))", "n_hi = int(np.count_nonzero(margin > eps))",
+     "test_oracle_geometry.py"),
+    ("geometry: coverage upper count ignores near misses", "oracle.geometry",
+     "n_hi[i] += bool((inside | (margin <= eps)).any())", "n_hi[i] += bool(inside.any())",
+     "test_oracle_geometry.py"),
+    ("geometry: inside margin takes the farthest face", "oracle.geometry",
+     "m_in = np.minimum(np.minimum(du, dv), dz)", "m_in = np.maximum(np.maximum(du, dv), dz)",
+     "test_oracle_geometry.py"),
+    ("multiwarp: marginal landings not marked unsure", "oracle.slabs",
+     "                if margin <= eps:\n                    for (x, y) in cand:",
+     "                if margin < -1.0:\n                    for (x, y) in cand:",
+     "test_oracle_slabs.py"),
+    ("multiwarp: candidates only the landing cell", "oracle.slabs",
+     "xs = {math.floor(pu - du), math.floor(pu), math.floor(pu + du)}", "xs = {math.floor(pu)}",
+     "test_oracle_slabs.py"),
+    ("multiwarp: median of the first two samples", "oracle.slabs",
+     "zq[y, x] = np.float32(np.median(np.asarray(vals, dtype=np.float64)))",
+     "zq[y, x] = np.float32(np.mean(np.asarray(vals[:2], dtype=np.float64)))",
+     "test_oracle_slabs.py"),
+    # ---- audit pooling
+    ("audit: R_geo averaged per row", "oracle.audit",
+     "R_geo=c[1] / n_pos if n_pos else float(\"nan\"),",
+     "R_geo=float(np.nanmean(np.asarray(counts).reshape(-1, 6)[:, 1] / np.maximum(np.asarray(counts).reshape(-1, 6)[:, 0], 1))),",
+     "test_oracle_audit.py"),
+    ("audit: changed counted against the model's top-50", "oracle.audit",
+     "len(pos & f_fuse), len(f_fuse - a_fuse)", "len(pos & f_fuse), len(f_fuse - a_geo)",
+     "test_oracle_audit.py"),
+    # ---- Gilbert construction details
+    ("gilbert: minor halves not made even", "oracle.gilbert",
+     "if abs(hbx + hby) % 2 == 1 and n_minor > 2:", "if False:", "test_oracle_gilbert.py"),
+    ("thw: neighbours from the Gilbert blocks", "oracle.gilbert",
+     'order = {"gilbert": global_order, "thw": thw_linear_order}[layout]',
+     'order = {"gilbert": global_order, "thw": global_order}[layout]', "test_oracle_gilbert.py"),
+    # ---- importance / route details
+    ("route: reserved range off by one", "oracle.route",
+     "reserved = list(range(prev_begin, prev_begin + prev_count))",
+     "reserved = list(range(prev_begin, prev_begin + prev_count - 1))", "test_oracle_route.py"),
+    ("route: budget left unsorted", "oracle.route",
+     "return sorted(budget), extras, info", "return budget, extras, info", "test_oracle_route.py"),
+    ("attention: scale applied after the max", "oracle.attention",
+     """    x = (q @ k.T) * scale
+    m = x.max(axis=1, keepdims=True)
+    e = np.exp(x - m)
+    l = e.sum(axis=1, keepdims=True)
+    O = (e @ v) / l""",
+     """    x = (q @ k.T)
+    m = x.max(axis=1, keepdims=True)
+    e = np.exp((x - m) * scale)
+    l = e.sum(axis=1, keepdims=True)
+    O = (e @ v) / l""", "test_oracle_attention.py"),
 ]
 
 

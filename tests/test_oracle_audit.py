@@ -124,3 +124,20 @@ def test_positive_overlap_is_strictly_above_tau():
     g[0, 5:8] = np.nextafter(np.float32(0.1), np.float32(1))
     c = oa.audit(p, g, ort.Params(tau=0.1), 5, 8)
     assert c[0, 0, 0] == 3
+
+
+def test_metrics_pool_rows_and_changed_is_against_the_model_top_k():
+    # R_geo is a ratio of sums over rows (10 / 12), not a mean of per-row
+    # ratios (0.5)
+    c = np.zeros((2, 6), dtype=np.int64)
+    c[0, :2] = [10, 10]
+    c[1, :2] = [2, 0]
+    assert oa.metrics(c, 143).R_geo == 10 / 12
+    # lambda = 0 with the defaults (top-50 for R_geo, top-80 for the fusion
+    # rows): the fused top-80 is the model's top-80, nothing changes
+    rng = np.random.default_rng(8)
+    M = 143
+    p = _softmax_rows(rng.standard_normal((1, 4, M)))
+    g = _g_audit(rng, 4, M)
+    c = oa.audit(p, g, ort.Params(lam=0.0))
+    assert np.all(c[..., 5] == 0) and oa.metrics(c, M).changed == 0.0

@@ -169,3 +169,12 @@ def test_covered_when_rho_equals_eta():
     uvz[0, :, 2] = [4.0, 4.0, 9.0, 9.0]
     rho, cov = geo.coverage([cam()], [0], uvz, [0], [SLAB], [1], eta=0.5)
     assert rho.tolist() == [0.5] and cov.tolist() == [1]
+
+
+def test_coverage_upper_count_holds_tokens_just_outside():
+    # a token exactly on the far face u = u1 is outside (the rectangle is
+    # half-open) but within the marginal distance: n_hi counts it, n does not
+    c = cam()
+    uvz = np.array([[[6.0, 3.0, 4.0]], [[3.0, 6.0, 4.0]], [[7.0, 3.0, 4.0]]], dtype=np.float32)
+    n, lo, hi = geo.coverage_bounds([c], [0, 0, 0], uvz, [0], [SLAB], [1])
+    assert n.tolist() == [0, 0, 0] and lo.tolist() == [0, 0, 0] and hi.tolist() == [1, 1, 0]

@@ -179,3 +179,15 @@ def test_slab_needs_exactly_n_min_reliable_samples():
                                     osl.SlabParams(s=1, n_min=4))
     assert valid.tolist() == [1, 0]
     assert slab[0].tolist() == [0.0, 4.0, 0.0, 1.0, 2.0, 2.0]
+
+
+def test_a_marginal_landing_makes_both_neighbours_unsure():
+    # one valid sample, moved half a token sideways: it lands exactly on the
+    # edge between target tokens 2 and 3 of row 1, so either may receive it
+    # in another precision; nothing else is unsure
+    H, W, Z = 4, 8, 4.0
+    d = np.zeros((1, H, W), dtype=np.float32)
+    d[0, 1, 3] = Z
+    src, tgt = cam(), cam(C=(0.5, 0.0, 0.0))
+    zq, unsure = osl.multiwarp_bounds([src, tgt], d, [0], 1, H, W, s=1, k_warp=1)
+    assert sorted(zip(*np.nonzero(unsure))) == [(1, 2), (1, 3)]
