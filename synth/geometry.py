@@ -114,3 +114,55 @@ def pack_slabs(slab: np.ndarray, cam: np.ndarray, valid=None) -> np.ndarray:
     out[:, 6] = cam
     out[:, 7] = 1 if valid is None else valid
     return out
+
+
+def random_pose_scene(seed: int, N: int, M: int, b: int = 64, frame_hw=(32, 48),
+                      n_cams: int = 6, max_angle: float = 0.6,
+                      p_invalid: float = 0.1) -> Scene:
+    """A scene with arbitrary camera poses, for fuzzing the geometry.
+
+    ``n_cams`` cameras with rotations about random axes by up to
+    ``max_angle`` radians (Rodrigues' formula), centres in [-1, 1]^3, focal
+    lengths 20-60 and principal points near the frame centre; N query and M
+    history slabs with random rectangles (1-16 tokens a side) of random
+    cameras, depth intervals starting in [1, 8] with widths 0.2-4; each
+    query block's b tokens sit in its rectangle with depths around its
+    interval (about 10 % holes).  Seeded numpy, no projection arithmetic.
+    """
+    rng = np.random.default_rng(seed)
+    fh, fw = frame_hw
+    cams = np.zeros((n_cams, 16), dtype=np.float32)
+    for k in range(n_cams):
+        axis = rng.standard_normal(3)
+        axis /= np.linalg.norm(axis)
+        ang = rng.uniform(-max_angle, max_angle)
+        Kx = np.array([[0.0, -axis[2], axis[1]], [axis[2], 0.0, -axis[0]],
+                       [-axis[1], axis[0], 0.0]])
+        R = np.eye(3) + np.sin(ang) * Kx + (1.0 - np.cos(ang)) * Kx @ Kx
+        C = rng.uniform(-1.0, 1.0, size=3)
+        f = rng.uniform(20.0, 60.0, size=2)
+        cx, cy = fw / 2.0 + rng.uniform(-4.0, 4.0), fh / 2.0 + rng.uniform(-3.0, 3.0)
+        cams[k] = [f[0], f[1], cx, cy, *R.reshape(-1), *C]
+
+    def slabs(n):
+        w = rng.integers(1, 17, size=n)
+        h = rng.integers(1, 17, size=n)
+        u0 = rng.integers(0, fw - w + 1)
+        v0 = rng.integers(0, fh - h + 1)
+        zlo = rng.uniform(1.0, 8.0, size=n)
+        zhi = zlo + rng.uniform(0.2, 4.0, size=n)
+        sl = np.stack([u0, u0 + w, v0, v0 + h, zlo, zhi], 1).astype(np.float32)
+        return sl, rng.integers(0, n_cams, size=n).astype(np.int32)
+
+    h_slab, h_cam = slabs(M)
+    h_valid = (rng.random(M) >= p_invalid).astype(np.int32)
+    q_slab, q_cam = slabs(N)
+    q_uvz = np.zeros((N, b, 3), dtype=np.float32)
+    for i in range(N):
+        u0, u1, v0, v1, zlo, zhi = (float(x) for x in q_slab[i])
+        q_uvz[i, :, 0] = rng.uniform(u0, u1, size=b)
+        q_uvz[i, :, 1] = rng.uniform(v0, v1, size=b)
+        z = rng.uniform(zlo - 0.3, zhi + 0.3, size=b)
+        z[rng.random(b) < 0.1] = 0.0
+        q_uvz[i, :, 2] = z
+    return Scene(cams, q_slab, q_cam, q_uvz, h_slab, h_cam, h_valid)

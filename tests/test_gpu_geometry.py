@@ -155,3 +155,22 @@ def test_host_validation(lib):
     cov = torch.zeros(2, dtype=torch.uint8, device="cuda")
     with pytest.raises(rbs.VeloxError):
         rbs.velox_coverage(cams, cams.shape[0], qs, uvz, 2, 129, hs, 4, 0.9, rho, cov, st)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_random_poses_overlap_and_coverage(lib, seed):
+    # arbitrary rotations (up to 0.6 rad about random axes), focal lengths,
+    # principal points, rectangles and depth ranges: g and the covered counts
+    # against the fp64 oracle under the marginal-decision rule
+    from synth.geometry import random_pose_scene
+    s = random_pose_scene(seed, 7, 60, b=64)
+    G = (2, 4, 8)[seed % 3]
+    g, st = _overlap(s, G)
+    assert st == 0
+    ref, lo, hi = _bounds(s, G)
+    check_g_bounds(g, ref, lo, hi)
+    rho, cov, st = _coverage(s, eta=0.5)
+    assert st == 0
+    n, nlo, nhi = geo.coverage_bounds(s.cams, s.q_cam, s.q_uvz, s.h_cam, s.h_slab, s.h_valid)
+    check_coverage_bounds(rho, cov, n, nlo, nhi, 64, 0.5)
+
