@@ -145,8 +145,8 @@ def random_pose_scene(seed: int, N: int, M: int, b: int = 64, frame_hw=(32, 48),
         cams[k] = [f[0], f[1], cx, cy, *R.reshape(-1), *C]
 
     def slabs(n):
-        w = rng.integers(1, 17, size=n)
-        h = rng.integers(1, 17, size=n)
+        w = rng.integers(1, min(16, fw) + 1, size=n)
+        h = rng.integers(1, min(16, fh) + 1, size=n)
         u0 = rng.integers(0, fw - w + 1)
         v0 = rng.integers(0, fh - h + 1)
         zlo = rng.uniform(1.0, 8.0, size=n)
@@ -166,3 +166,14 @@ def random_pose_scene(seed: int, N: int, M: int, b: int = 64, frame_hw=(32, 48),
         z[rng.random(b) < 0.1] = 0.0
         q_uvz[i, :, 2] = z
     return Scene(cams, q_slab, q_cam, q_uvz, h_slab, h_cam, h_valid)
+
+
+def random_depth_maps(seed: int, n_frames: int, H: int, W: int, s: int = 1,
+                      p_hole: float = 0.1) -> np.ndarray:
+    """[n_frames][H s][W s] fp32 depths drawn uniformly from [2, 8], a
+    fraction p_hole of them 0 (no depth): source maps for fuzzing the
+    multiwarp with the cameras of random_pose_scene."""
+    rng = np.random.default_rng(seed)
+    d = rng.uniform(2.0, 8.0, size=(n_frames, H * s, W * s)).astype(np.float32)
+    d[rng.random(d.shape) < p_hole] = 0.0
+    return d

@@ -203,3 +203,20 @@ def test_geometry_chain_depth_to_g_and_coverage(lib):
     check_g_bounds(g.cpu().numpy().astype(np.float64), g_ref, g_lo, g_hi)
     n, n_lo, n_hi = geo.coverage_bounds(r.cams, qc, quvz, hc, hs, hv)
     check_coverage_bounds(rho.cpu().numpy(), cov.cpu().numpy(), n, n_lo, n_hi, b, 0.9)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_multiwarp_random_poses(lib, seed):
+    # sources and target from cameras rotated up to 0.6 rad about random
+    # axes with different intrinsics; depths uniform in [2, 8] with holes
+    from synth.geometry import random_depth_maps, random_pose_scene
+    H, W = 8, 16
+    s = 1 + seed % 2
+    k = 1 + seed % 3
+    cams = random_pose_scene(seed, 1, 1, frame_hw=(H, W), n_cams=5).cams
+    src = [4, 3, 2, 1]                        # newest first
+    depth = random_depth_maps(seed, len(src), H, W, s)
+    zq, st = _gpu_multiwarp(cams, depth, src, [0], H, W, s, k)
+    assert st == 0
+    ref, unsure = osl.multiwarp_bounds(cams, depth, src, 0, H, W, s, k)
+    check_multiwarp(zq[0], ref, unsure)
