@@ -138,3 +138,51 @@ def test_thw_neighbours_bit_exact(lib, T, H, W, b, nc, qc, first, M):
         assert c[i] == len(ref[i])
         assert got[i, :c[i]].tolist() == ref[i]
         assert np.all(got[i, c[i]:] == -1)
+
+
+def _random_lattices(seed, n):
+    """Seeded supported lattices: W >= H, not (W odd and H even), b a
+    divisor of T H W (>= 4 keeps the oracle's neighbour search quick)."""
+    r = np.random.default_rng(seed)
+    out = []
+    while len(out) < n:
+        T = int(r.integers(1, 4))
+        H = int(r.integers(1, 13))
+        W = int(r.integers(H, 25))
+        if W % 2 == 1 and H % 2 == 0:
+            continue
+        cells = T * H * W
+        divs = [d for d in range(4, min(cells, 256) + 1) if cells % d == 0]
+        if not divs:
+            continue
+        b = int(r.choice(divs))
+        nc = int(r.integers(2, 5))
+        out.append((T, H, W, b, nc))
+    return out
+
+
+@pytest.mark.parametrize("T,H,W,b,nc", _random_lattices(20261203, 20))
+def test_random_lattices_order_and_neighbours_bit_exact(lib, T, H, W, b, nc):
+    n = nc * T * H * W
+    rank = torch.full((n,), -7, dtype=torch.int32, device="cuda")
+    cell = torch.full((n,), -7, dtype=torch.int32, device="cuda")
+    block = torch.full((n,), -7, dtype=torch.int32, device="cuda")
+    N = T * H * W // b
+    qc, M = nc - 1, (nc - 1) * N
+    S_max = 256
+    ids = torch.full((N, S_max), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.full((N,), -7, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lib.velox_gilbert_order(T, H, W, nc, b, qc, 0, M, rank_of_cell=rank, cell_of_rank=cell,
+                            block_of_cell=block, nbr_ids=ids, nbr_cnt=cnt, S_max=S_max,
+                            dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    r_ref, c_ref, b_ref = gilbert.global_order(T, H, W, nc, b)
+    assert np.array_equal(rank.cpu().numpy(), r_ref)
+    assert np.array_equal(cell.cpu().numpy(), c_ref)
+    assert np.array_equal(block.cpu().numpy(), b_ref)
+    ref = gilbert.neighbour_blocks(T, H, W, nc, b, qc, 0, M)
+    ids, cnt = ids.cpu().numpy(), cnt.cpu().numpy()
+    for i in range(N):
+        assert cnt[i] == len(ref[i]) and ids[i, :cnt[i]].tolist() == ref[i]
