@@ -103,12 +103,14 @@ def make_inputs(wl: Workload, device="cpu", out: Optional[Inputs] = None,
                   ref_ids=ref.to(device))
 
 
-def make_current(wl: Workload, device="cpu"):
-    """K and V of the chunk being generated, [H][N*b][d] bf16 ~ N(0, 1): the
-    second phase of two-phase attention (its own seed, disjoint from Q/K/V)."""
+def make_current(wl: Workload, device="cpu", n_blocks: Optional[int] = None):
+    """K and V of the chunk being generated, [H][n*b][d] bf16 ~ N(0, 1) with
+    n = n_blocks (default: the workload's N query blocks): the second phase
+    of two-phase attention (its own seed, disjoint from Q/K/V)."""
     device = torch.device(device)
     gen = torch.Generator(device=device).manual_seed(wl.seed * 7 + 5)
-    shape = (wl.heads, wl.n_q_blocks * wl.b, wl.d)
+    n = wl.n_q_blocks if n_blocks is None else n_blocks
+    shape = (wl.heads, n * wl.b, wl.d)
     Kc = torch.empty(shape, dtype=torch.bfloat16, device=device).normal_(generator=gen)
     Vc = torch.empty(shape, dtype=torch.bfloat16, device=device).normal_(generator=gen)
     return Kc, Vc

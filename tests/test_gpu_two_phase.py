@@ -102,3 +102,23 @@ def test_two_phase_chunk48_sampled_rows(lib):
     assert st == 0
     rows = [(0, 0), (17, 31), (39, 47), (8, 5)]
     assert_attention_close(O, lse, _oracle(inp, Kc, Vc, rows, lambda h, i: routes[(h, i)]))
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_two_phase_random_cases(lib, seed):
+    # N_cur independent of N, random route lengths (empty ones included),
+    # the longest-first row order
+    r = np.random.default_rng(3000 + seed)
+    H, N, M = int(r.integers(1, 4)), int(r.integers(1, 6)), int(r.integers(1, 40))
+    n_cur = int(r.integers(1, 7))
+    wl = small(H, N, M, 0, layer=seed)
+    inp = make_inputs(wl, "cuda")
+    Kc, Vc = make_current(wl, "cuda", n_blocks=n_cur)
+    R = int(r.integers(1, M + 1))
+    rid, rln, routes = _routes(H, N, M, R, 3100 + seed)
+    order = torch.empty(H * N, dtype=torch.int32, device="cuda")
+    rbs.velox_route_schedule(rln, H * N, R, order)
+    O, lse, st = _run(inp, Kc, Vc, rid, rln, R, order)
+    assert st == 0
+    ref = _oracle(inp, Kc, Vc, sorted(routes), lambda h, i: routes[(h, i)])
+    assert_attention_close(O, lse, ref)
