@@ -69,3 +69,37 @@ def test_attention_random_cases(lib, seed):
     ref = attention_rows(inp.Q, inp.K, inp.V, sorted(routes), lambda h, i: routes[(h, i)],
                          scale)
     assert_attention_close(O, lse, ref)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_attention_random_medium_cases(lib, seed):
+    # hundreds to thousands of history blocks, routes of up to 300 tiles,
+    # up to 2 heads x 24 query blocks; 6 sampled rows per case
+    r = np.random.default_rng(4000 + seed)
+    H, N, M = int(r.integers(1, 3)), int(r.integers(4, 25)), int(r.integers(100, 3001))
+    inp = make_inputs(small(H, N, M, 0, layer=seed), "cuda")
+    R_max = int(r.integers(1, min(M, 300) + 1))
+    ids = torch.full((H, N, R_max), -1, dtype=torch.int32)
+    ln = torch.zeros(H, N, dtype=torch.int32)
+    routes = {}
+    for h in range(H):
+        for i in range(N):
+            k = int(r.integers(0, R_max + 1))
+            sel = r.choice(M, size=k, replace=False).tolist()
+            ids[h, i, :k] = torch.tensor(sel, dtype=torch.int32)
+            ln[h, i] = k
+            routes[(h, i)] = sel
+    O = torch.full((H, N * 128, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((H, N * 128), float("nan"), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    order = torch.empty(H * N, dtype=torch.int32, device="cuda")
+    rid, rln = ids.cuda(), ln.cuda()
+    rbs.velox_route_schedule(rln, H * N, R_max, order)
+    rbs.velox_block_sparse_attn(inp.Q, inp.K, inp.V, rid, rln, R_max, H, N, M, 128, 128, 0.0,
+                                O, lse, st, row_order=order)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rows = sorted(routes)
+    pick = [rows[int(x)] for x in r.choice(len(rows), size=min(6, len(rows)), replace=False)]
+    ref = attention_rows(inp.Q, inp.K, inp.V, sorted(pick), lambda h, i: routes[(h, i)])
+    assert_attention_close(O, lse, ref)
