@@ -142,8 +142,9 @@ __global__ void __launch_bounds__(256) logits_kernel(const float *__restrict__ q
 
 // Fused K pooling + logits.  Grid-stride over chunks of 8 * per_warp key
 // blocks of one head (chunk c: head c / cpr, blocks (c % cpr) * 8 * per_warp
-// ..), 256 threads, grid sized to the resident capacity; per_warp is 8 unless
-// H * M is too small to give every CTA slot a chunk.
+// ..), 256 threads, grid sized to the resident capacity (two CTAs per SM:
+// the registers of 16 loads in flight per lane plus the dot products);
+// per_warp is the count whose busiest CTA streams the fewest blocks.
 // Warp w of a CTA streams the per_warp consecutive key blocks r0 + w per_warp
 // .. with no block-level barrier after the qbar load.  After the half-warp
 // exchange both halves hold the 8 channel sums of lane (l & 15); half-warp 0
@@ -151,11 +152,15 @@ __global__ void __launch_bounds__(256) logits_kernel(const float *__restrict__ q
 // 1, 3, 5, ..., each as 8 products plus a 16-lane shuffle reduction, staged
 // in the warp's own [N][8] shared-memory slice and written out row by row
 // (8 consecutive logits = 32 bytes per row) once the warp's blocks are done.
+// The warp's load stream does not stop for those products: the first 16
+// loads of block k are issued before the products of block k - 1, which run
+// while they are in flight.  Each sum and each product is formed in the same
+// order as without the overlap.
 constexpr int kFusedMaxN = 96;
 constexpr int kFusedWarps = 8;
 constexpr int kFusedPerWarp = 8;  // most key blocks per warp (the staging width)
 
-__global__ void __launch_bounds__(256) pool_logits_kernel(const uint16_t *__restrict__ K,
+__global__ void __launch_bounds__(kFusedWarps * 32) pool_logits_kernel(const uint16_t *__restrict__ K,
                                                           const float *__restrict__ qbar, int H,
                                                           int N, int M, float scale,
                                                           int per_warp, float *__restrict__ p) {
@@ -175,38 +180,49 @@ __global__ void __launch_bounds__(256) pool_logits_kernel(const uint16_t *__rest
     fsm[e] = reinterpret_cast<const float4 *>(qbar + (size_t)h * N * D)[e];
   __syncthreads();
   const int rw = (c - h * cpr) * per_cta + warp * per_warp;  // first block of the warp
-  for (int k = 0; k < per_warp; ++k) {
-    const int rb = rw + k;
-    if (rb >= M) break;  // uniform across the warp
-    float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    const uint16_t *src = K + ((size_t)h * M + rb) * BT * D + row0 * D + col;
-#pragma unroll 1
-    for (int r = 0; r < BT / 2; r += 16) {
-      uint4 v[16];
+  const int nb = min(per_warp, M - rw);  // this warp's blocks (none past M)
+  float sum[8];  // channel sums of the previous block (both half-warps)
+  for (int k = 0; nb > 0 && k <= nb; ++k) {
+    const bool more = k < nb;  // uniform across the warp
+    const uint16_t *src = K + ((size_t)h * M + rw + (more ? k : 0)) * BT * D + row0 * D + col;
+    uint4 v[16];
+    if (more) {
 #pragma unroll
-      for (int q = 0; q < 16; ++q) v[q] = ld_stream(src + (size_t)(r + q) * 2 * D);
+      for (int q = 0; q < 16; ++q) v[q] = ld_stream(src + (size_t)q * 2 * D);
+    }
+    if (k > 0) {
+      // logits of block k - 1; same trip count in both half-warps (the
+      // shuffles span the whole warp)
+      for (int ii = 0; ii < (N + 1) / 2; ++ii) {
+        const int i = 2 * ii + row0;
+        const int iq = i < N ? i : N - 1;  // odd N: half-warp 1 repeats a row, unused
+        const float4 q0 = *reinterpret_cast<const float4 *>(qs + iq * D + col);
+        const float4 q1 = *reinterpret_cast<const float4 *>(qs + iq * D + col + 4);
+        float d = q0.x * sum[0];
+        d = fmaf(q0.y, sum[1], d); d = fmaf(q0.z, sum[2], d); d = fmaf(q0.w, sum[3], d);
+        d = fmaf(q1.x, sum[4], d); d = fmaf(q1.y, sum[5], d); d = fmaf(q1.z, sum[6], d);
+        d = fmaf(q1.w, sum[7], d);
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+        if ((lane & 15) == 0 && i < N) lg[i * kFusedPerWarp + k - 1] = d * cs;
+      }
+    }
+    if (more) {
+      float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
       for (int q = 0; q < 16; ++q) acc8(a, v[q]);
-    }
+#pragma unroll 1
+      for (int r = 16; r < BT / 2; r += 16) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q) a[q] += __shfl_xor_sync(0xffffffffu, a[q], 16);
-    // same trip count in both half-warps (the shuffles span the whole warp)
-    for (int ii = 0; ii < (N + 1) / 2; ++ii) {
-      const int i = 2 * ii + row0;
-      const int iq = i < N ? i : N - 1;  // odd N: half-warp 1 repeats a row, unused
-      const float4 q0 = *reinterpret_cast<const float4 *>(qs + iq * D + col);
-      const float4 q1 = *reinterpret_cast<const float4 *>(qs + iq * D + col + 4);
-      float d = q0.x * a[0];
-      d = fmaf(q0.y, a[1], d); d = fmaf(q0.z, a[2], d); d = fmaf(q0.w, a[3], d);
-      d = fmaf(q1.x, a[4], d); d = fmaf(q1.y, a[5], d); d = fmaf(q1.z, a[6], d);
-      d = fmaf(q1.w, a[7], d);
+        for (int q = 0; q < 16; ++q) v[q] = ld_stream(src + (size_t)(r + q) * 2 * D);
 #pragma unroll
-      for (int off = 8; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-      if ((lane & 15) == 0 && i < N) lg[i * kFusedPerWarp + k] = d * cs;
+        for (int q = 0; q < 16; ++q) acc8(a, v[q]);
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) sum[q] = a[q] + __shfl_xor_sync(0xffffffffu, a[q], 16);
     }
   }
   __syncwarp();
-  const int nb = min(per_warp, M - rw);
   for (int e = lane; e < N * kFusedPerWarp; e += 32) {
     const int i = e / kFusedPerWarp, k = e - i * kFusedPerWarp;
     if (k < nb) p[((size_t)h * N + i) * M + rw + k] = lg[e];
@@ -286,13 +302,21 @@ cudaError_t launch_importance(const uint16_t *Q, const uint16_t *K, int H, int N
                                (int)smem);
       if (e != cudaSuccess) return e;
     }
-    int per_sm = (int)((220 * 1024) / (smem + 1024));
-    per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
+    // CTA slots: what the registers and shared memory let reside per SM
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pool_logits_kernel,
+                                                      kFusedWarps * 32, smem);
+    if (e != cudaSuccess) return e;
+    per_sm = per_sm < 1 ? 1 : per_sm;
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
     // key blocks per warp: the count (1..8) whose busiest CTA streams the
     // fewest blocks, i.e. ceil(chunks / slots) * per_warp smallest, the larger
-    // count on ties -- 8 at the chunk-48 shape, fewer when a few heads would
-    // leave CTA slots empty
-    const long long slots = 148LL * per_sm;
+    // count on ties (with 2 CTAs on each of 148 SMs and 2256 key blocks: 3 at
+    // 40 heads, 5 at 20, 8 at 16, 5 at 10 and 5)
+    const long long slots = (long long)sms * per_sm;
     int per_warp = kFusedPerWarp;
     long long best = -1;
     for (int pw = kFusedPerWarp; pw >= 1; --pw) {
@@ -305,7 +329,8 @@ cudaError_t launch_importance(const uint16_t *Q, const uint16_t *K, int H, int N
     }
     const int chunks = H * ((M + kFusedWarps * per_warp - 1) / (kFusedWarps * per_warp));
     const int grid_f = chunks < slots ? chunks : (int)slots;
-    pool_logits_kernel<<<grid_f, 256, smem, stream>>>(K, qbar, H, N, M, scale, per_warp, p);
+    pool_logits_kernel<<<grid_f, kFusedWarps * 32, smem, stream>>>(K, qbar, H, N, M, scale,
+                                                                   per_warp, p);
   } else {
     dim3 lg((M + LG_R - 1) / LG_R, H);
     logits_kernel<<<lg, 256, 0, stream>>>(qbar, kbar, N, M, scale, p);
