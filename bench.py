@@ -672,6 +672,66 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
+def run_dense_vs_cudnn(args):
+    """Dense attention over the whole chunk-48 history (H=40, 6,144 query
+    tokens, 288,768 cache tokens, d=128): this library's dense mode
+    (route_ids = NULL) against torch's scaled_dot_product_attention on its
+    cuDNN backend (NVIDIA's fused attention for this GPU) and on its
+    FlashAttention-2 backend, the same bf16 tensors, each trial after a
+    cool-down, the kinds interleaved.  Context for the attention kernel's
+    roofline fraction; not the bench line."""
+    import time
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    from routed_block_sparse_b200.pipeline import layer_for
+    from synth import config, make_inputs
+
+    wl = config(3)
+    inp = make_inputs(wl, "cuda")
+    layer = layer_for(wl)
+    H, N, M, b, d = wl.heads, wl.n_q_blocks, wl.n_kv_blocks, 128, 128
+    q = inp.Q.view(1, H, N * b, d)
+    k = inp.K.view(1, H, M * b, d)
+    v = inp.V.view(1, H, M * b, d)
+    flops = 4.0 * H * (N * b) * (M * b) * d
+    kinds = {"velox_dense": lambda: layer.attend(inp.Q, inp.K, inp.V, dense=True)}
+    for name, be in (("cudnn", SDPBackend.CUDNN_ATTENTION),
+                     ("flash2", SDPBackend.FLASH_ATTENTION)):
+        def call(be=be):
+            with sdpa_kernel([be]):
+                return F.scaled_dot_product_attention(q, k, v)
+        kinds[name] = call
+    out = {"workload": "dense attention, chunk-48 layer over its whole history",
+           "heads": H, "q_tokens": N * b, "kv_tokens": M * b, "head_dim": d,
+           "tflop_per_call": flops / 1e12}
+    layer.attend(inp.Q, inp.K, inp.V, dense=True)
+    mine = layer.O.view(1, H, N * b, d).float()
+    for name in list(kinds):
+        if name == "velox_dense":
+            continue
+        try:
+            o = kinds[name]()
+            torch.cuda.synchronize()
+            out[f"{name}_max_abs_vs_velox"] = float((o.float() - mine).abs().max())
+            del o
+        except RuntimeError as e:  # backend not built for this GPU or shape
+            out[f"{name}_error"] = str(e)[:160]
+            del kinds[name]
+    del mine
+    best = {n: float("inf") for n in kinds}
+    for _ in range(3):
+        for name, fn in kinds.items():
+            torch.cuda.synchronize()
+            time.sleep(1.0)
+            best[name] = min(best[name], _time_us(fn, reps=5, warm=2))
+    for name, us in best.items():
+        out[f"{name}_ms"] = us / 1e3
+        out[f"{name}_tflops"] = flops / (us * 1e-6) / 1e12
+    if "cudnn" in best:
+        out["velox_dense_vs_cudnn"] = best["cudnn"] / best["velox_dense"]
+    print(json.dumps(out), flush=True)
+
+
 def _time_us(fn, reps=50, warm=3):
     for _ in range(warm):
         fn()
@@ -1049,6 +1109,8 @@ def main():
     ap.add_argument("--layout", default="both", choices=["both", "gilbert", "thw"])
     ap.add_argument("--qk", default="both", choices=["both", "random", "positional"],
                     help="--layouts input recipe: random N(0,1) Q/K or positional Q/K")
+    ap.add_argument("--dense-vs-cudnn", action="store_true",
+                    help="dense attention: this library against torch SDPA (cuDNN, FA2)")
     ap.add_argument("--heads", type=int, default=0,
                     help="run a reduced head count (profiler captures only)")
     args = ap.parse_args()
@@ -1066,6 +1128,9 @@ def main():
     try:
         if args.sweep:
             run_sweep(args)
+            return
+        if args.dense_vs_cudnn:
+            run_dense_vs_cudnn(args)
             return
         if args.geometry:
             run_geometry(args)

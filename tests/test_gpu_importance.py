@@ -54,6 +54,18 @@ def test_importance_ragged_shapes(lib, H, N, M):
     _check(p, oracle_importance(inp.Q, inp.K, range(H), 1.0))
 
 
+@pytest.mark.parametrize("H,M", [(1, 300), (8, 300), (16, 300), (24, 300), (32, 300),
+                                 (39, 300), (19, 777), (17, 1000)])
+def test_importance_every_chunk_width(lib, H, M):
+    # The fused kernel streams chunks of 8 * w key blocks (w per warp, 1..8,
+    # picked from H and M).  On a 148-SM part with two CTAs per SM these
+    # shapes pick w = 1, 2, ..., 8 in turn, and each ends on a partial chunk
+    # (warps with fewer than w blocks and warps with none).  N = 5 is odd.
+    inp = make_inputs(small(H, 5, M, 0), "cuda")
+    p = _run(lib, inp, 1.0)
+    _check(p, oracle_importance(inp.Q, inp.K, range(H), 1.0))
+
+
 def test_importance_peaked_logits(lib):
     # large scale: logits of order 100, rows nearly one-hot.  An fp32 logit
     # carries an absolute error of about |logit| * 2^-23 ~ 1e-5, which turns
