@@ -13,8 +13,10 @@
 //                        one head's key blocks with that head's qbar in
 //                        shared memory; each warp pools one block and its two
 //                        half-warps dot the mean with half of the query rows
-//                        each; logits are staged in shared memory and written
-//                        into p row-contiguously.  No key means touch memory.
+//                        each, while the warp's loads of its next block are
+//                        in flight; logits are staged in shared memory and
+//                        written into p row-contiguously.  No key means touch
+//                        memory.
 //   softmax_kernel       per (head, query block) row: max, sum of exp,
 //                        normalise, in place.
 // When N > kFusedMaxN the key means go through the workspace instead
