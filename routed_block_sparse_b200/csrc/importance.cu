@@ -17,8 +17,11 @@
 //                        in flight; logits are staged in shared memory and
 //                        written into p row-contiguously.  No key means touch
 //                        memory.
-//   softmax_kernel       per (head, query block) row: max, sum of exp,
-//                        normalise, in place.
+//   softmax_row_kernel   per (head, query block) row, one warp with the row
+//                        in registers: max, exponentials and their sum,
+//                        normalise, in place (softmax_kernel, a CTA per row
+//                        with an online max/sum merge, for rows that do not
+//                        fit).
 // When N > kFusedMaxN the key means go through the workspace instead
 // (pool_kernel on K, then logits_kernel).
 #include "common.cuh"
@@ -240,7 +243,8 @@ __device__ __forceinline__ void merge_ms(float &m, float &s, float m2, float s2)
   m = mm;
 }
 
-// One CTA per (h, i) row of M logits, in place.
+// One CTA per (h, i) row of M logits, in place; for rows the one-warp kernel
+// below cannot hold (M above 4096, not a multiple of 4, or p not 16-byte aligned).
 __global__ void __launch_bounds__(256) softmax_kernel(float *__restrict__ p, int M) {
   __shared__ float sm[8], ss[8];
   float *row = p + (size_t)blockIdx.x * M;
@@ -276,6 +280,49 @@ __global__ void __launch_bounds__(256) softmax_kernel(float *__restrict__ p, int
   __syncthreads();
   const float gm = sm[0], inv = 1.0f / ss[0];
   for (int r = threadIdx.x; r < M; r += blockDim.x) row[r] = expf(row[r] - gm) * inv;
+}
+
+// One warp per (head, query block) row with the whole row in registers:
+// VMAX float4 per lane, so rows of up to 128 * VMAX logits (M a multiple of 4,
+// rows 16-byte aligned).  The row is read once and written once; each logit
+// takes one exponential.
+template <int VMAX>
+__global__ void __launch_bounds__(256) softmax_row_kernel(float *__restrict__ p, int M,
+                                                         int rows) {
+  const int wrow = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wrow >= rows) return;  // uniform across the warp
+  float4 *row = reinterpret_cast<float4 *>(p + (size_t)wrow * M);
+  const int n4 = M >> 2;
+  float4 x[VMAX];
+#pragma unroll
+  for (int j = 0; j < VMAX; ++j) {
+    const int c = lane + 32 * j;
+    x[j] = c < n4 ? row[c] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+  }
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < VMAX; ++j) m = fmaxf(m, fmaxf(fmaxf(x[j].x, x[j].y), fmaxf(x[j].z, x[j].w)));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < VMAX; ++j) {
+    x[j].x = expf(x[j].x - m);  // padding: exp(-inf) = 0
+    x[j].y = expf(x[j].y - m);
+    x[j].z = expf(x[j].z - m);
+    x[j].w = expf(x[j].w - m);
+    s += (x[j].x + x[j].y) + (x[j].z + x[j].w);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  const float inv = 1.0f / s;
+#pragma unroll
+  for (int j = 0; j < VMAX; ++j) {
+    const int c = lane + 32 * j;
+    if (c < n4)
+      row[c] = make_float4(x[j].x * inv, x[j].y * inv, x[j].z * inv, x[j].w * inv);
+  }
 }
 
 }  // namespace
@@ -339,7 +386,17 @@ cudaError_t launch_importance(const uint16_t *Q, const uint16_t *K, int H, int N
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  softmax_kernel<<<H * N, 256, 0, stream>>>(p, M);
+  const int rows = H * N;
+  const int rgrid = (rows + 7) / 8;  // eight rows (warps) per CTA
+  if ((M & 3) != 0 || (reinterpret_cast<uintptr_t>(p) & 15u) != 0 || M > 128 * 32) {
+    softmax_kernel<<<rows, 256, 0, stream>>>(p, M);
+  } else if (M <= 128 * 8) {
+    softmax_row_kernel<8><<<rgrid, 256, 0, stream>>>(p, M, rows);
+  } else if (M <= 128 * 18) {
+    softmax_row_kernel<18><<<rgrid, 256, 0, stream>>>(p, M, rows);
+  } else {
+    softmax_row_kernel<32><<<rgrid, 256, 0, stream>>>(p, M, rows);
+  }
   return cudaGetLastError();
 }
 
