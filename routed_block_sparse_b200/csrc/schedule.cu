@@ -11,6 +11,7 @@ namespace velox {
 namespace {
 
 constexpr int kThreads = 1024;
+constexpr int kKeepRows = 8192;  // rows whose bins stay in shared memory
 
 __global__ void __launch_bounds__(kThreads) schedule_kernel(const int32_t *__restrict__ route_len,
                                                             int rows, int R_max,
@@ -18,12 +19,18 @@ __global__ void __launch_bounds__(kThreads) schedule_kernel(const int32_t *__res
   extern __shared__ int bins[];  // R_max + 1 counters, bin k = length R_max - k
   __shared__ int s_warp[kThreads / 32];
   const int nb = R_max + 1;
+  // the bin of every row, kept for the placement pass when it fits (one warp
+  // walks the rows in order there, and a global load per step would set its
+  // pace)
+  int *row_bin = bins + nb;
+  const bool keep = rows <= kKeepRows;
   for (int k = threadIdx.x; k < nb; k += kThreads) bins[k] = 0;
   __syncthreads();
   for (int r = threadIdx.x; r < rows; r += kThreads) {
     int L = route_len[r];
     L = (L < 0 || L > R_max) ? 0 : L;
     atomicAdd(&bins[R_max - L], 1);
+    if (keep) row_bin[r] = R_max - L;
   }
   __syncthreads();
   // exclusive scan of the bins (thread t owns a contiguous run)
@@ -53,9 +60,16 @@ __global__ void __launch_bounds__(kThreads) schedule_kernel(const int32_t *__res
   if (warp == 0) {
     for (int base = 0; base < rows; base += 32) {
       const int r = base + lane;
-      int L = r < rows ? route_len[r] : -1;
-      if (r < rows && (L < 0 || L > R_max)) L = 0;
-      const int bin = R_max - L;
+      int bin = -1;
+      if (r < rows) {
+        if (keep) {
+          bin = row_bin[r];
+        } else {
+          int L = route_len[r];
+          L = (L < 0 || L > R_max) ? 0 : L;
+          bin = R_max - L;
+        }
+      }
       const unsigned peers = __match_any_sync(0xffffffffu, bin);
       const int rank = __popc(peers & ((1u << lane) - 1u));
       int start = 0;
@@ -74,7 +88,7 @@ __global__ void __launch_bounds__(kThreads) schedule_kernel(const int32_t *__res
 
 cudaError_t launch_schedule(const int32_t *route_len, int rows, int R_max, int32_t *row_order,
                             cudaStream_t stream) {
-  const size_t smem = (size_t)(R_max + 1) * sizeof(int);
+  const size_t smem = ((size_t)(R_max + 1) + (rows <= kKeepRows ? (size_t)rows : 0)) * sizeof(int);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(schedule_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -17,7 +17,8 @@ from synth import make_inputs
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("rows,R_max", [(1, 1), (37, 5), (1920, 214), (5000, 4096)])
+@pytest.mark.parametrize("rows,R_max", [(1, 1), (37, 5), (1920, 214), (5000, 4096), (8192, 300),
+                                        (9000, 300)])
 def test_schedule_is_the_stable_longest_first_order(lib, rows, R_max):
     r = np.random.default_rng(rows)
     L = r.integers(0, R_max + 1, rows).astype(np.int32)
