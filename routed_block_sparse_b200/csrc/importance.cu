@@ -7,7 +7,7 @@
 // Three launches:
 //   pool_kernel          query blocks: fp32 means qbar [H][N][d] into the
 //                        workspace.  One warp per 128 x 128 bf16 block,
-//                        16-byte non-caching loads, 8 loads in flight per lane.
+//                        16-byte non-caching loads, 16 in flight per lane.
 //   pool_logits_kernel   streams K once (the HBM-bound part: 2.96 GB at the
 //                        chunk-48 shape).  A CTA takes a contiguous range of
 //                        one head's key blocks with that head's qbar in
@@ -50,7 +50,7 @@ __device__ __forceinline__ void acc8(float (&a)[8], const uint4 &v) {
 // Unit u < n_q: block u of Q (means to qbar); else block u - n_q of K (to kbar).
 // Rows of a block are 256 bytes = 16 lanes x 16 bytes: lanes 0-15 take even
 // rows, lanes 16-31 odd rows; each lane sums 8 channels over 64 rows.
-__global__ void __launch_bounds__(256) pool_kernel(const uint16_t *__restrict__ Q,
+__global__ void __launch_bounds__(256, 1) pool_kernel(const uint16_t *__restrict__ Q,
                                                    const uint16_t *__restrict__ K, int n_q,
                                                    int n_units, float *__restrict__ qbar,
                                                    float *__restrict__ kbar) {
@@ -72,12 +72,12 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t *__restrict__ 
     float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     const uint16_t *p = src + row0 * D + col;
 #pragma unroll 1
-    for (int r = 0; r < BT / 2; r += 8) {
-      uint4 v[8];
+    for (int r = 0; r < BT / 2; r += 16) {
+      uint4 v[16];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) v[k] = ld_stream(p + (size_t)(r + k) * 2 * D);
+      for (int k = 0; k < 16; ++k) v[k] = ld_stream(p + (size_t)(r + k) * 2 * D);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) acc8(a, v[k]);
+      for (int k = 0; k < 16; ++k) acc8(a, v[k]);
     }
 #pragma unroll
     for (int k = 0; k < 8; ++k) a[k] += __shfl_xor_sync(0xffffffffu, a[k], 16);
