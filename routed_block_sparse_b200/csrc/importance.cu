@@ -49,7 +49,10 @@ __device__ __forceinline__ void acc8(float (&a)[8], const uint4 &v) {
 
 // Unit u < n_q: block u of Q (means to qbar); else block u - n_q of K (to kbar).
 // Rows of a block are 256 bytes = 16 lanes x 16 bytes: lanes 0-15 take even
-// rows, lanes 16-31 odd rows; each lane sums 8 channels over 64 rows.
+// rows, lanes 16-31 odd rows; each lane sums 8 channels over 64 rows, 16
+// loads in flight at a time (the occupancy floor of one CTA leaves the
+// compiler the registers for all 16; a chunk-48 launch has under two CTAs per
+// SM anyway).
 __global__ void __launch_bounds__(256, 1) pool_kernel(const uint16_t *__restrict__ Q,
                                                    const uint16_t *__restrict__ K, int n_q,
                                                    int n_units, float *__restrict__ qbar,
