@@ -49,8 +49,13 @@ def test_importance_chunk48_every_head(lib):
     _check(p, oracle_importance(inp.Q, inp.K, range(inp.wl.heads), 1.0))
 
 
-@pytest.mark.parametrize("H,N,M", [(1, 1, 1), (2, 3, 65), (3, 17, 130), (1, 40, 200)])
+@pytest.mark.parametrize("H,N,M", [(1, 1, 1), (2, 3, 65), (3, 17, 130), (1, 40, 200),
+                                   (1, 2, 1024), (1, 2, 1028), (2, 3, 2304), (1, 2, 2308),
+                                   (2, 3, 4096)])
 def test_importance_ragged_shapes(lib, H, N, M):
+    # M = 1024 / 2304 / 4096 are the largest rows of each register-resident
+    # softmax width (8, 18, 32 float4 per lane), 1028 and 2308 the smallest
+    # above them; M not a multiple of 4 takes the CTA-per-row softmax
     inp = make_inputs(small(H, N, M, 0), "cuda")
     p = _run(lib, inp, 1.0)
     _check(p, oracle_importance(inp.Q, inp.K, range(H), 1.0))
