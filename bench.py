@@ -15,8 +15,10 @@ across them (strong scaling; `--shard layers` gives every rank its own layer
 instead); there is no data-path collective.  Per-call times, the roofline of
 the attention kernel (with the SM clock measured from the GPU beside the
 attention calls: the driver's sampled clock does not show the power
-limiter), an end-to-end number through host buffers and the CPU oracle
-baseline are added.
+limiter), two end-to-end numbers through host buffers (`e2e`: every input
+of the step copied in each step; `e2e_rollout`: the KV cache kept in HBM and
+only what a rollout's step brings in copied) and the CPU oracle baseline are
+added.
 """
 
 from __future__ import annotations
@@ -536,6 +538,7 @@ def run_velox(args, world, rank, local):
     # end to end through the public API with host buffers
     if args.e2e_steps > 0:
         line["e2e"] = _e2e(args, wl, inp, layer, dev, stream, flops_step, world)
+        line["e2e_rollout"] = _e2e_rollout(args, wl, inp, layer, dev, stream, flops_step, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r = cpu_oracle_sample(inp)
         line["cpu_baseline"] = {"value": flops_step / r["step_s"] / 1e12, "unit": UNIT,
@@ -633,6 +636,63 @@ def _e2e(args, wl, inp, layer, dev, stream, flops_step, world):
     val = _sum_over_ranks(flops_step, world) / (ms * 1e-3) / 1e12
     return {"value": val, "unit": UNIT, "ms_per_step": ms, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h}
+
+
+def _e2e_rollout(args, wl, inp, layer, dev, stream, flops_step, world):
+    """The step as a rollout runs it, through the public API with the KV cache
+    kept in HBM: per step, pinned host -> device copies of the current chunk's
+    Q, of the previous chunk's K and V (written into the cache slots that
+    chunk occupies: one copy per head and tensor), of g and of the coverage
+    flags; the neighbour table and the four calls; O and lse back to the
+    host.  Each history chunk crosses the host link once, when it joins the
+    cache; the synthetic steps re-send the same previous chunk into the same
+    slots, so the cache does not change between them.  Timed with CUDA
+    events."""
+    # token rows of the previous chunk's blocks (K and V are [H][M*b][d])
+    t0, t1 = wl.prev_begin * wl.b, (wl.prev_begin + wl.prev_count) * wl.b
+    H = wl.heads
+    q_h = inp.Q.cpu().pin_memory()
+    g_h = inp.g.cpu().pin_memory()
+    c_h = inp.covered.cpu().pin_memory()
+    k_new = inp.K[:, t0:t1].cpu().pin_memory()
+    v_new = inp.V[:, t0:t1].cpu().pin_memory()
+    out_O = torch.empty_like(layer.O, device="cpu").pin_memory()
+    out_lse = torch.empty_like(layer.lse, device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, g_h, c_h, k_new, v_new))
+    d2h = out_O.numel() * out_O.element_size() + out_lse.numel() * out_lse.element_size()
+    T, Hl, Wl = wl.lattice
+    import routed_block_sparse_b200 as rbs
+
+    def one():
+        inp.Q.copy_(q_h, non_blocking=True)
+        for h in range(H):
+            inp.K[h, t0:t1].copy_(k_new[h], non_blocking=True)
+            inp.V[h, t0:t1].copy_(v_new[h], non_blocking=True)
+        inp.g.copy_(g_h, non_blocking=True)
+        inp.covered.copy_(c_h, non_blocking=True)
+        rbs.velox_gilbert_order(T, Hl, Wl, wl.n_chunks, wl.b, wl.q_chunk, wl.cache_first_block,
+                                wl.n_kv_blocks, nbr_ids=layer.nbr_ids, nbr_cnt=layer.nbr_cnt,
+                                S_max=layer.S_max, dev_status=layer.dev_status, stream=stream)
+        layer.forward(inp.Q, inp.K, inp.V, inp.g, inp.covered, stream)
+        out_O.copy_(layer.O, non_blocking=True)
+        out_lse.copy_(layer.lse, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    z = torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        one()
+    z.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = _max_over_ranks(a.elapsed_time(z) / args.e2e_steps, world)
+    val = _sum_over_ranks(flops_step, world) / (ms * 1e-3) / 1e12
+    return {"value": val, "unit": UNIT, "ms_per_step": ms, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h,
+            "inputs": "current chunk's Q, previous chunk's K/V into its cache slots, g, "
+                      "coverage flags; the rest of the KV cache stays in HBM"}
 
 
 def run_sweep(args):
