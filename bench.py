@@ -647,7 +647,7 @@ def _e2e_rollout(args, wl, inp, layer, dev, stream, flops_step, world):
     host.  Each history chunk crosses the host link once, when it joins the
     cache; the synthetic steps re-send the same previous chunk into the same
     slots, so the cache does not change between them.  Timed with CUDA
-    events."""
+    events on the launching stream, which every copy stream joins."""
     # token rows of the previous chunk's blocks (K and V are [H][M*b][d])
     t0, t1 = wl.prev_begin * wl.b, (wl.prev_begin + wl.prev_count) * wl.b
     H = wl.heads
@@ -663,19 +663,37 @@ def _e2e_rollout(args, wl, inp, layer, dev, stream, flops_step, world):
     T, Hl, Wl = wl.lattice
     import routed_block_sparse_b200 as rbs
 
+    # What the importance needs (Q, K) crosses first; g, the flags and V follow
+    # on a copy stream while the importance runs, and the route build and the
+    # attention wait only for what they read.
+    copy = torch.cuda.Stream(dev)
+    ev_k, ev_g, ev_v = (torch.cuda.Event() for _ in range(3))
+
     def one():
-        inp.Q.copy_(q_h, non_blocking=True)
-        for h in range(H):
-            inp.K[h, t0:t1].copy_(k_new[h], non_blocking=True)
-            inp.V[h, t0:t1].copy_(v_new[h], non_blocking=True)
-        inp.g.copy_(g_h, non_blocking=True)
-        inp.covered.copy_(c_h, non_blocking=True)
+        with torch.cuda.stream(stream):
+            inp.Q.copy_(q_h, non_blocking=True)
+            for h in range(H):
+                inp.K[h, t0:t1].copy_(k_new[h], non_blocking=True)
+        ev_k.record(stream)
+        copy.wait_event(ev_k)  # also orders V's slots after the last step's attention
+        with torch.cuda.stream(copy):
+            inp.g.copy_(g_h, non_blocking=True)
+            inp.covered.copy_(c_h, non_blocking=True)
+            ev_g.record(copy)
+            for h in range(H):
+                inp.V[h, t0:t1].copy_(v_new[h], non_blocking=True)
+            ev_v.record(copy)
         rbs.velox_gilbert_order(T, Hl, Wl, wl.n_chunks, wl.b, wl.q_chunk, wl.cache_first_block,
                                 wl.n_kv_blocks, nbr_ids=layer.nbr_ids, nbr_cnt=layer.nbr_cnt,
                                 S_max=layer.S_max, dev_status=layer.dev_status, stream=stream)
-        layer.forward(inp.Q, inp.K, inp.V, inp.g, inp.covered, stream)
-        out_O.copy_(layer.O, non_blocking=True)
-        out_lse.copy_(layer.lse, non_blocking=True)
+        layer.importance(inp.Q, inp.K, stream)
+        stream.wait_event(ev_g)
+        layer.route(inp.g, inp.covered, stream=stream)
+        stream.wait_event(ev_v)
+        layer.attend(inp.Q, inp.K, inp.V, stream=stream)
+        with torch.cuda.stream(stream):
+            out_O.copy_(layer.O, non_blocking=True)
+            out_lse.copy_(layer.lse, non_blocking=True)
 
     one()
     torch.cuda.synchronize(dev)
