@@ -603,27 +603,58 @@ def _graph_replay(step, steps, dev):
 
 def _e2e(args, wl, inp, layer, dev, stream, flops_step, world):
     """Per step: pinned host -> device copy of Q, K, V, g, covered; the four
-    calls; device -> host copy of O and lse.  Timed with CUDA events."""
+    calls; device -> host copy of O and lse.  The heads are independent
+    through the whole path, so the step runs in head groups: a copy stream
+    sends g, the flags and then each group's Q, K and V, and the launching
+    stream runs a group's importance, route build and attention as soon as
+    its inputs have landed, and sends its O and lse back while later groups
+    are still crossing.  Timed with CUDA events on the launching stream,
+    which the copy stream joins."""
+    from dataclasses import replace
+    from routed_block_sparse_b200.pipeline import layer_for
+    import routed_block_sparse_b200 as rbs
+
     host = {k: getattr(inp, k).cpu().pin_memory() for k in ("Q", "K", "V", "g", "covered")}
     out_O = torch.empty_like(layer.O, device="cpu").pin_memory()
     out_lse = torch.empty_like(layer.lse, device="cpu").pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_O.numel() * out_O.element_size() + out_lse.numel() * out_lse.element_size()
     T, Hl, Wl = wl.lattice
-    import routed_block_sparse_b200 as rbs
+    H = wl.heads
+    n_groups = min(8, H)
+    bounds = [(H * k // n_groups, H * (k + 1) // n_groups) for k in range(n_groups)]
+    layers = [layer_for(replace(wl, heads=h1 - h0), device=dev) for h0, h1 in bounds]
+    for lg in layers[1:]:  # one neighbour table per step, read by every group
+        lg.nbr_ids, lg.nbr_cnt = layers[0].nbr_ids, layers[0].nbr_cnt
+    copy = torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in bounds]
+    ev_gc = torch.cuda.Event()
 
     def one():
-        for k, t in host.items():
-            getattr(inp, k).copy_(t, non_blocking=True)
+        copy.wait_stream(stream)  # the last step is done with every input
+        with torch.cuda.stream(copy):
+            inp.g.copy_(host["g"], non_blocking=True)
+            inp.covered.copy_(host["covered"], non_blocking=True)
+            ev_gc.record(copy)
+            for (h0, h1), ev in zip(bounds, ev_in):
+                for k in ("Q", "K", "V"):
+                    getattr(inp, k)[h0:h1].copy_(host[k][h0:h1], non_blocking=True)
+                ev.record(copy)
+        l0 = layers[0]
         rbs.velox_gilbert_order(T, Hl, Wl, wl.n_chunks, wl.b, wl.q_chunk, wl.cache_first_block,
-                                wl.n_kv_blocks, nbr_ids=layer.nbr_ids, nbr_cnt=layer.nbr_cnt,
-                                S_max=layer.S_max, dev_status=layer.dev_status, stream=stream)
-        layer.forward(inp.Q, inp.K, inp.V, inp.g, inp.covered, stream)
-        out_O.copy_(layer.O, non_blocking=True)
-        out_lse.copy_(layer.lse, non_blocking=True)
+                                wl.n_kv_blocks, nbr_ids=l0.nbr_ids, nbr_cnt=l0.nbr_cnt,
+                                S_max=l0.S_max, dev_status=l0.dev_status, stream=stream)
+        stream.wait_event(ev_gc)
+        for (h0, h1), ev, lg in zip(bounds, ev_in, layers):
+            stream.wait_event(ev)
+            lg.forward(inp.Q[h0:h1], inp.K[h0:h1], inp.V[h0:h1], inp.g, inp.covered, stream)
+            with torch.cuda.stream(stream):
+                out_O[h0:h1].copy_(lg.O, non_blocking=True)
+                out_lse[h0:h1].copy_(lg.lse, non_blocking=True)
 
     one()
     torch.cuda.synchronize(dev)
+    status = max(int(lg.status()) for lg in layers)
     a = torch.cuda.Event(enable_timing=True)
     z = torch.cuda.Event(enable_timing=True)
     _barrier(world)
@@ -635,7 +666,7 @@ def _e2e(args, wl, inp, layer, dev, stream, flops_step, world):
     ms = _max_over_ranks(a.elapsed_time(z) / args.e2e_steps, world)
     val = _sum_over_ranks(flops_step, world) / (ms * 1e-3) / 1e12
     return {"value": val, "unit": UNIT, "ms_per_step": ms, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h}
+            "d2h_bytes_per_step": d2h, "head_groups": n_groups, "dev_status": status}
 
 
 def _e2e_rollout(args, wl, inp, layer, dev, stream, flops_step, world):
