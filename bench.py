@@ -601,28 +601,31 @@ def _graph_replay(step, steps, dev):
         return {"error": str(e)[:200]}
 
 
-def _e2e(args, wl, inp, layer, dev, stream, flops_step, world):
-    """Per step: pinned host -> device copy of Q, K, V, g, covered; the four
-    calls; device -> host copy of O and lse.  The heads are independent
-    through the whole path, so the step runs in head groups: a copy stream
-    sends g, the flags and then each group's Q, K and V, and the launching
-    stream runs a group's importance, route build and attention as soon as
-    its inputs have landed, and sends its O and lse back while later groups
-    are still crossing.  Timed with CUDA events on the launching stream,
-    which the copy stream joins."""
+def _e2e_grouped(args, wl, inp, layer, dev, stream, flops_step, world, group_copies):
+    """One end-to-end step through the public API, timed with CUDA events on
+    the launching stream: g and the coverage flags, then each head group's
+    inputs (group_copies(h0, h1): (device view, pinned host tensor) pairs)
+    cross on a copy stream; the launching stream runs the neighbour table,
+    then a group's importance, route build and attention as soon as its
+    inputs have landed, and sends its O and lse back while later groups are
+    still crossing.  The heads are independent through the whole path, so
+    this is the same step as one call over all heads."""
     from dataclasses import replace
     from routed_block_sparse_b200.pipeline import layer_for
     import routed_block_sparse_b200 as rbs
 
-    host = {k: getattr(inp, k).cpu().pin_memory() for k in ("Q", "K", "V", "g", "covered")}
+    g_h = inp.g.cpu().pin_memory()
+    c_h = inp.covered.cpu().pin_memory()
     out_O = torch.empty_like(layer.O, device="cpu").pin_memory()
     out_lse = torch.empty_like(layer.lse, device="cpu").pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_O.numel() * out_O.element_size() + out_lse.numel() * out_lse.element_size()
     T, Hl, Wl = wl.lattice
     H = wl.heads
     n_groups = min(8, H)
     bounds = [(H * k // n_groups, H * (k + 1) // n_groups) for k in range(n_groups)]
+    plans = [group_copies(h0, h1) for h0, h1 in bounds]
+    h2d = g_h.numel() * g_h.element_size() + c_h.numel() * c_h.element_size() + sum(
+        src.numel() * src.element_size() for plan in plans for _, src in plan)
+    d2h = out_O.numel() * out_O.element_size() + out_lse.numel() * out_lse.element_size()
     layers = [layer_for(replace(wl, heads=h1 - h0), device=dev) for h0, h1 in bounds]
     for lg in layers[1:]:  # one neighbour table per step, read by every group
         lg.nbr_ids, lg.nbr_cnt = layers[0].nbr_ids, layers[0].nbr_cnt
@@ -633,12 +636,12 @@ def _e2e(args, wl, inp, layer, dev, stream, flops_step, world):
     def one():
         copy.wait_stream(stream)  # the last step is done with every input
         with torch.cuda.stream(copy):
-            inp.g.copy_(host["g"], non_blocking=True)
-            inp.covered.copy_(host["covered"], non_blocking=True)
+            inp.g.copy_(g_h, non_blocking=True)
+            inp.covered.copy_(c_h, non_blocking=True)
             ev_gc.record(copy)
-            for (h0, h1), ev in zip(bounds, ev_in):
-                for k in ("Q", "K", "V"):
-                    getattr(inp, k)[h0:h1].copy_(host[k][h0:h1], non_blocking=True)
+            for plan, ev in zip(plans, ev_in):
+                for dst, src in plan:
+                    dst.copy_(src, non_blocking=True)
                 ev.record(copy)
         l0 = layers[0]
         rbs.velox_gilbert_order(T, Hl, Wl, wl.n_chunks, wl.b, wl.q_chunk, wl.cache_first_block,
@@ -669,79 +672,41 @@ def _e2e(args, wl, inp, layer, dev, stream, flops_step, world):
             "d2h_bytes_per_step": d2h, "head_groups": n_groups, "dev_status": status}
 
 
+def _e2e(args, wl, inp, layer, dev, stream, flops_step, world):
+    """Every input of the step (Q, K, V, g, the coverage flags) copied from
+    pinned host memory each step; O and lse copied back."""
+    host = {k: getattr(inp, k).cpu().pin_memory() for k in ("Q", "K", "V")}
+
+    def copies(h0, h1):
+        return [(getattr(inp, k)[h0:h1], host[k][h0:h1]) for k in ("Q", "K", "V")]
+
+    return _e2e_grouped(args, wl, inp, layer, dev, stream, flops_step, world, copies)
+
+
 def _e2e_rollout(args, wl, inp, layer, dev, stream, flops_step, world):
-    """The step as a rollout runs it, through the public API with the KV cache
-    kept in HBM: per step, pinned host -> device copies of the current chunk's
-    Q, of the previous chunk's K and V (written into the cache slots that
-    chunk occupies: one copy per head and tensor), of g and of the coverage
-    flags; the neighbour table and the four calls; O and lse back to the
-    host.  Each history chunk crosses the host link once, when it joins the
-    cache; the synthetic steps re-send the same previous chunk into the same
-    slots, so the cache does not change between them.  Timed with CUDA
-    events on the launching stream, which every copy stream joins."""
+    """The step as a rollout runs it, with the KV cache kept in HBM: each step
+    copies in the current chunk's Q, the previous chunk's K and V (into the
+    cache slots that chunk occupies: one copy per head and tensor), g and the
+    coverage flags, and copies O and lse out.  Each history chunk crosses the
+    host link once, when it joins the cache; the synthetic steps re-send the
+    same previous chunk into the same slots, so the cache does not change
+    between them."""
     # token rows of the previous chunk's blocks (K and V are [H][M*b][d])
     t0, t1 = wl.prev_begin * wl.b, (wl.prev_begin + wl.prev_count) * wl.b
-    H = wl.heads
     q_h = inp.Q.cpu().pin_memory()
-    g_h = inp.g.cpu().pin_memory()
-    c_h = inp.covered.cpu().pin_memory()
     k_new = inp.K[:, t0:t1].cpu().pin_memory()
     v_new = inp.V[:, t0:t1].cpu().pin_memory()
-    out_O = torch.empty_like(layer.O, device="cpu").pin_memory()
-    out_lse = torch.empty_like(layer.lse, device="cpu").pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (q_h, g_h, c_h, k_new, v_new))
-    d2h = out_O.numel() * out_O.element_size() + out_lse.numel() * out_lse.element_size()
-    T, Hl, Wl = wl.lattice
-    import routed_block_sparse_b200 as rbs
 
-    # What the importance needs (Q, K) crosses first; g, the flags and V follow
-    # on a copy stream while the importance runs, and the route build and the
-    # attention wait only for what they read.
-    copy = torch.cuda.Stream(dev)
-    ev_k, ev_g, ev_v = (torch.cuda.Event() for _ in range(3))
+    def copies(h0, h1):
+        plan = [(inp.Q[h0:h1], q_h[h0:h1])]
+        for h in range(h0, h1):
+            plan += [(inp.K[h, t0:t1], k_new[h]), (inp.V[h, t0:t1], v_new[h])]
+        return plan
 
-    def one():
-        with torch.cuda.stream(stream):
-            inp.Q.copy_(q_h, non_blocking=True)
-            for h in range(H):
-                inp.K[h, t0:t1].copy_(k_new[h], non_blocking=True)
-        ev_k.record(stream)
-        copy.wait_event(ev_k)  # also orders V's slots after the last step's attention
-        with torch.cuda.stream(copy):
-            inp.g.copy_(g_h, non_blocking=True)
-            inp.covered.copy_(c_h, non_blocking=True)
-            ev_g.record(copy)
-            for h in range(H):
-                inp.V[h, t0:t1].copy_(v_new[h], non_blocking=True)
-            ev_v.record(copy)
-        rbs.velox_gilbert_order(T, Hl, Wl, wl.n_chunks, wl.b, wl.q_chunk, wl.cache_first_block,
-                                wl.n_kv_blocks, nbr_ids=layer.nbr_ids, nbr_cnt=layer.nbr_cnt,
-                                S_max=layer.S_max, dev_status=layer.dev_status, stream=stream)
-        layer.importance(inp.Q, inp.K, stream)
-        stream.wait_event(ev_g)
-        layer.route(inp.g, inp.covered, stream=stream)
-        stream.wait_event(ev_v)
-        layer.attend(inp.Q, inp.K, inp.V, stream=stream)
-        with torch.cuda.stream(stream):
-            out_O.copy_(layer.O, non_blocking=True)
-            out_lse.copy_(layer.lse, non_blocking=True)
-
-    one()
-    torch.cuda.synchronize(dev)
-    a = torch.cuda.Event(enable_timing=True)
-    z = torch.cuda.Event(enable_timing=True)
-    _barrier(world)
-    a.record(stream)
-    for _ in range(args.e2e_steps):
-        one()
-    z.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = _max_over_ranks(a.elapsed_time(z) / args.e2e_steps, world)
-    val = _sum_over_ranks(flops_step, world) / (ms * 1e-3) / 1e12
-    return {"value": val, "unit": UNIT, "ms_per_step": ms, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h,
-            "inputs": "current chunk's Q, previous chunk's K/V into its cache slots, g, "
-                      "coverage flags; the rest of the KV cache stays in HBM"}
+    out = _e2e_grouped(args, wl, inp, layer, dev, stream, flops_step, world, copies)
+    out["inputs"] = ("current chunk's Q, previous chunk's K/V into its cache slots, g, "
+                     "coverage flags; the rest of the KV cache stays in HBM")
+    return out
 
 
 def run_sweep(args):
