@@ -607,8 +607,8 @@ def _e2e_grouped(args, wl, inp, layer, dev, stream, flops_step, world, group_cop
     inputs (group_copies(h0, h1): (device view, pinned host tensor) pairs)
     cross on a copy stream; the launching stream runs the neighbour table,
     then a group's importance, route build and attention as soon as its
-    inputs have landed, and sends its O and lse back while later groups are
-    still crossing.  The heads are independent through the whole path, so
+    inputs have landed, and a third stream sends the group's O and lse back
+    while later groups are still crossing or computing.  The heads are independent through the whole path, so
     this is the same step as one call over all heads."""
     from dataclasses import replace
     from routed_block_sparse_b200.pipeline import layer_for
@@ -629,8 +629,10 @@ def _e2e_grouped(args, wl, inp, layer, dev, stream, flops_step, world, group_cop
     layers = [layer_for(replace(wl, heads=h1 - h0), device=dev) for h0, h1 in bounds]
     for lg in layers[1:]:  # one neighbour table per step, read by every group
         lg.nbr_ids, lg.nbr_cnt = layers[0].nbr_ids, layers[0].nbr_cnt
-    copy = torch.cuda.Stream(dev)
+    copy = torch.cuda.Stream(dev)   # host -> device
+    back = torch.cuda.Stream(dev)   # device -> host
     ev_in = [torch.cuda.Event() for _ in bounds]
+    ev_out = [torch.cuda.Event() for _ in bounds]
     ev_gc = torch.cuda.Event()
 
     def one():
@@ -648,12 +650,15 @@ def _e2e_grouped(args, wl, inp, layer, dev, stream, flops_step, world, group_cop
                                 wl.n_kv_blocks, nbr_ids=l0.nbr_ids, nbr_cnt=l0.nbr_cnt,
                                 S_max=l0.S_max, dev_status=l0.dev_status, stream=stream)
         stream.wait_event(ev_gc)
-        for (h0, h1), ev, lg in zip(bounds, ev_in, layers):
+        for (h0, h1), ev, done, lg in zip(bounds, ev_in, ev_out, layers):
             stream.wait_event(ev)
             lg.forward(inp.Q[h0:h1], inp.K[h0:h1], inp.V[h0:h1], inp.g, inp.covered, stream)
-            with torch.cuda.stream(stream):
+            done.record(stream)
+            back.wait_event(done)
+            with torch.cuda.stream(back):
                 out_O[h0:h1].copy_(lg.O, non_blocking=True)
                 out_lse[h0:h1].copy_(lg.lse, non_blocking=True)
+        stream.wait_stream(back)  # the step ends when O and lse are on the host
 
     one()
     torch.cuda.synchronize(dev)
