@@ -620,7 +620,7 @@ def _e2e_grouped(args, wl, inp, layer, dev, stream, flops_step, world, group_cop
     out_lse = torch.empty_like(layer.lse, device="cpu").pin_memory()
     T, Hl, Wl = wl.lattice
     H = wl.heads
-    n_groups = min(8, H)
+    n_groups = max(1, min(args.e2e_groups, H))
     bounds = [(H * k // n_groups, H * (k + 1) // n_groups) for k in range(n_groups)]
     plans = [group_copies(h0, h1) for h0, h1 in bounds]
     h2d = g_h.numel() * g_h.element_size() + c_h.numel() * c_h.element_size() + sum(
@@ -691,8 +691,8 @@ def _e2e(args, wl, inp, layer, dev, stream, flops_step, world):
 def _e2e_rollout(args, wl, inp, layer, dev, stream, flops_step, world):
     """The step as a rollout runs it, with the KV cache kept in HBM: each step
     copies in the current chunk's Q, the previous chunk's K and V (into the
-    cache slots that chunk occupies: one copy per head and tensor), g and the
-    coverage flags, and copies O and lse out.  Each history chunk crosses the
+    cache slots that chunk occupies), g and the coverage flags, and copies O
+    and lse out.  Each history chunk crosses the
     host link once, when it joins the cache; the synthetic steps re-send the
     same previous chunk into the same slots, so the cache does not change
     between them."""
@@ -703,10 +703,10 @@ def _e2e_rollout(args, wl, inp, layer, dev, stream, flops_step, world):
     v_new = inp.V[:, t0:t1].cpu().pin_memory()
 
     def copies(h0, h1):
-        plan = [(inp.Q[h0:h1], q_h[h0:h1])]
-        for h in range(h0, h1):
-            plan += [(inp.K[h, t0:t1], k_new[h]), (inp.V[h, t0:t1], v_new[h])]
-        return plan
+        # one copy per tensor and group: the slots of the group's heads are a
+        # strided view (torch stages it through a contiguous device buffer)
+        return [(inp.Q[h0:h1], q_h[h0:h1]), (inp.K[h0:h1, t0:t1], k_new[h0:h1]),
+                (inp.V[h0:h1, t0:t1], v_new[h0:h1])]
 
     out = _e2e_grouped(args, wl, inp, layer, dev, stream, flops_step, world, copies)
     out["inputs"] = ("current chunk's Q, previous chunk's K/V into its cache slots, g, "
@@ -1171,6 +1171,8 @@ def main():
                          "give every rank its own layer (weak scaling)")
     ap.add_argument("--impl", default="velox", choices=["velox", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-groups", type=int, default=8,
+                    help="head groups the end-to-end step pipelines its host copies over")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="history-length sweep: routed vs dense attention per M (extra lines)")
