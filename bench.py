@@ -621,7 +621,7 @@ def _e2e_grouped(args, wl, inp, layer, dev, stream, flops_step, world, group_cop
     T, Hl, Wl = wl.lattice
     H = wl.heads
     n_groups = max(1, min(args.e2e_groups, H))
-    bounds = [(H * k // n_groups, H * (k + 1) // n_groups) for k in range(n_groups)]
+    bounds = [head_range(k, n_groups, H) for k in range(n_groups)]  # as a head split
     plans = [group_copies(h0, h1) for h0, h1 in bounds]
     h2d = g_h.numel() * g_h.element_size() + c_h.numel() * c_h.element_size() + sum(
         src.numel() * src.element_size() for plan in plans for _, src in plan)
